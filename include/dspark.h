@@ -1,0 +1,218 @@
+/*
+ * dspark.h — C ABI of the DSpark confidence-scheduled verify step (libdspark.so, sm_100a).
+ *
+ * One verify round of confidence-scheduled speculative decoding, as the DSpark write-ups
+ * describe it, split into the steps that run on the GPU:
+ *
+ *   dspark_schedule        survival scan + greedy marginal-gain prefix scheduler + flattening
+ *   dspark_verify_attn_plan / dspark_verify_attn
+ *                          flattened ragged GQA attention of every verify token over its
+ *                          request's paged KV cache and its own earlier verify tokens
+ *   dspark_accept          exact acceptance rule, longest accepted prefix, residual / bonus
+ *                          resampling (or greedy verification)
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer argument is DEVICE memory owned by the caller, unless stated otherwise.
+ *     The library allocates nothing; scratch comes from caller-provided workspaces whose
+ *     size the *_workspace_bytes queries return.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and performs no host synchronisation, except dspark_read_error.
+ *   - Launch shapes depend only on capacity arguments (R, K, T_cap, V, ...), never on
+ *     device-resident results such as the scheduled token count, so one verify step can be
+ *     enqueued without reading anything back.
+ *   - Host-side argument validation returns a negative dspark_status before anything is
+ *     enqueued.  Bad device-resident data (a marker that does not match its request, a page
+ *     index outside the cache, a draft token outside the vocabulary, ...) sets bits in a
+ *     sticky per-device error word and the affected unit of work is skipped; kernels never
+ *     trap.  dspark_read_error returns and clears that word.
+ *   - Integer tensors are int32, row-major, densely packed.
+ *
+ * Sources (news write-ups of the DSpark paper; they describe the method, not an interface):
+ *   [P1] "刚融完500亿创始人亲自下场写代码DeepSeek不卷参数专治AI“嘴慢”" (mooersco.com),
+ *        section "2. 置信度调度验证" and the engineering table.
+ *   [P2] "DSpark 的 661% 提速，是真突破还是数字游戏？" (new-universe.cn), §一, §3.2.
+ *   [P3] "DeepSeek服务器不再卡顿！DSpark加速60% - 80%，推理成本降40%" (qwbw.cn),
+ *        sections "DSpark的神奇之处", "成本与质量的考量".
+ *   [P4] "DeepSeek DSpark speculative decoding 85 percent faster LLM inference"
+ *        (aibuzzwire.news), section "置信度计划、负载感知验证".
+ */
+#ifndef DSPARK_H
+#define DSPARK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *dspark_stream_t; /* identical to cudaStream_t */
+
+/* Return codes. */
+enum dspark_status {
+  DSPARK_OK = 0,
+  DSPARK_EINVAL = -1,        /* an argument is out of range or a required pointer is NULL */
+  DSPARK_ECUDA = -2,         /* a CUDA runtime call failed (launch, attribute, copy) */
+  DSPARK_EWORKSPACE = -3,    /* workspace NULL or smaller than the size query returned */
+  DSPARK_EDEVICE_DATA = -4,  /* dspark_read_error: device-resident data was invalid */
+  DSPARK_ETIMEOUT = -5,      /* reserved for bounded waits; no current kernel waits */
+  DSPARK_EUNSUPPORTED = -6   /* valid arguments outside what this build implements */
+};
+
+/* Element types of floating-point tensors. */
+enum dspark_dtype { DSPARK_F32 = 0, DSPARK_BF16 = 1 };
+
+/* Bits of the device error word (see dspark_read_error). */
+enum dspark_device_error {
+  DSPARK_DERR_CONF = 1 << 0,        /* a confidence outside [0, 1] or NaN (treated as 0) */
+  DSPARK_DERR_TABLE = 1 << 1,       /* a step-time entry <= 0 or NaN (scan stops there) */
+  DSPARK_DERR_KV_LEN = 1 << 2,      /* kv_len < 0 or beyond the block table */
+  DSPARK_DERR_PAGE = 1 << 3,        /* a block-table entry outside [0, num_pages) */
+  DSPARK_DERR_MARKER = 1 << 4,      /* markers[t] != (r, kv_len[r] + j) for token t = q_offsets[r]+j */
+  DSPARK_DERR_OFFSETS = 1 << 5,     /* q_offsets not a scan of 1 + verify_len within T_cap */
+  DSPARK_DERR_VERIFY_LEN = 1 << 6,  /* verify_len outside [0, K] */
+  DSPARK_DERR_TOKEN = 1 << 7,       /* a draft token outside [0, V) */
+  DSPARK_DERR_LOGITS = 1 << 8       /* a logit row whose maximum is not finite */
+};
+
+#define DSPARK_CONF_LAG 2             /* rounds between producing and consuming confidences */
+#define DSPARK_MAX_K 16               /* largest supported max-draft length K */
+#define DSPARK_MAX_CANDIDATES 16384   /* largest R*K the scheduler sorts in one CTA */
+
+/* Human-readable name of a dspark_status value (static storage, never NULL). */
+const char *dspark_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int dspark_version(void);
+
+/*
+ * dspark_schedule — pick every request's verify length for one round.
+ *
+ * Defined by [P2 §3.2] (inputs: load, per-position confidence, the engine's throughput curve),
+ * [P3 "DSpark的神奇之处"] (measure speed per batch size in advance; queue all requests' draft
+ * tokens by score, high to low; keep adding the next ones while the extra correct tokens pay
+ * for the extra time), [P4] (survival probabilities, global throughput maximisation) and
+ * [P1 engineering table] (the asynchronous scheduler reads confidences from two rounds
+ * earlier; all verify tokens are flattened and tagged with markers).  Computes:
+ *   S[r][k]   = c[r][0] * ... * c[r][k]       (float64, left to right), c = conf of round
+ *                                              max(round_idx - DSPARK_CONF_LAG, 0)
+ *   order     = all (r, k) by S descending, ties by k ascending then r ascending
+ *   f(n)      = (R + sum of the first n S in that order) / t_ms[R + n]
+ *   n*        = first n with f(n + 1) <= f(n), else min(R*K, T_cap - R)
+ *   verify_len[r] = number of r's candidates among the first n*  (a prefix of r's block)
+ *   q_offsets = exclusive scan of 1 + verify_len (length R + 1); *T_out = q_offsets[R]
+ *   markers[q_offsets[r] + j] = (r, kv_len[r] + j), j = 0..verify_len[r]
+ *
+ * conf_ring   float32 [ring_depth][R][K]; slot (i % ring_depth) holds the confidences
+ *             produced in round i.  ring_depth >= DSPARK_CONF_LAG + 1.
+ * round_idx   current round (>= 0); slot max(round_idx - 2, 0) % ring_depth is read.
+ * kv_len      int32 [R] cached tokens per request (positions of the verify tokens follow).
+ * t_ms        float64 [T_cap + 1], t_ms[T] = engine step time for T verify tokens (> 0).
+ * T_cap       capacity of the flattened batch, R <= T_cap.
+ * verify_len  out int32 [R]; q_offsets out int32 [R + 1]; markers out int32 [T_cap][2]
+ *             (entries past *T_out untouched); T_out out int32 [1]; objective out
+ *             float64 [1] = f(n*).
+ * Limits: 1 <= K <= DSPARK_MAX_K, R*K <= DSPARK_MAX_CANDIDATES.
+ */
+int dspark_schedule(const float *conf_ring, int ring_depth, int round_idx, int R, int K,
+                    const int32_t *kv_len, const double *t_ms, int T_cap,
+                    int32_t *verify_len, int32_t *q_offsets, int32_t *markers,
+                    int32_t *T_out, double *objective, dspark_stream_t stream);
+
+/*
+ * Workspace of the attention pair (plan + calls).  rows = (Hq / Hkv) * (K + 1) query rows
+ * per (request, KV head).  The workspace holds the work partition, per-segment arrival
+ * counters and split-KV partial results; it is reused by every attention call of a step.
+ */
+size_t dspark_verify_attn_workspace_bytes(int R, int Hq, int Hkv, int D, int K);
+
+/*
+ * dspark_verify_attn_plan — partition one step's attention work across the GPU.
+ *
+ * Work is the sequence of (request r, KV head g, KV tile) units in request-major order, each
+ * request contributing Hkv * max(1, ceil(kv_len[r] / 64)) units; the plan splits it into
+ * equal contiguous ranges, one per persistent CTA.  Call once per step after the schedule
+ * (the partition depends only on kv_len and the request count), before any
+ * dspark_verify_attn of that step; it also zeroes the workspace's arrival counters.
+ * kv_len int32 [R] (device); ws/ws_bytes as returned by the query above.
+ */
+int dspark_verify_attn_plan(const int32_t *kv_len, int R, int Hq, int Hkv, int D, int K,
+                            void *ws, size_t ws_bytes, dspark_stream_t stream);
+
+/*
+ * dspark_verify_attn — flattened ragged GQA attention of every verify token.
+ *
+ * Defined by [P1 engineering table, row "内核利用率暴跌"]: variable-length verification pads
+ * and unbalances standard decode kernels, so every verify token is an independent element
+ * and a marker tensor carries its sequence and position; [P2 §一] the target checks all draft
+ * tokens in one batched pass.  For verify token t = q_offsets[r] + j with markers[t] =
+ * (r, pos) and every query head h (KV head g = h / (Hq/Hkv)):
+ *   keys   = r's cached positions 0..kv_len[r]-1, then r's verify tokens i with
+ *            kv_len[r] + i <= pos (causal)
+ *   out[t][h] = softmax(scale * q[t][h] . keys) . values   (fp32 accumulation)
+ *
+ * q          [T_cap][Hq][D], k_new / v_new [T_cap][Hkv][D] — the verify tokens' own query,
+ *            key and value rows (post positional encoding), in flattened token order.
+ * kv_pages   [num_pages][2][Hkv][page_size][D] paged cache: index 0 = K, 1 = V; one
+ *            page holds page_size consecutive positions of one request.
+ * block_table int32 [R][max_pages]: physical page of each request's i-th page.
+ * kv_len     int32 [R]; markers int32 [T_cap][2]; q_offsets int32 [R + 1] (from the schedule;
+ *            only rows t < q_offsets[R] are read or written).
+ * out        [T_cap][Hq][D], same dtype as the inputs.
+ * dtype      DSPARK_BF16 (tensor-core path when D == 128 and page_size % 64 == 0) or
+ *            DSPARK_F32; scale is usually 1/sqrt(D).
+ * Limits: 1 <= D <= 256 with D % 8 == 0, Hq % Hkv == 0, (Hq/Hkv)*(K+1) <= 128.
+ */
+int dspark_verify_attn(const void *q, const void *k_new, const void *v_new,
+                       const void *kv_pages, int64_t num_pages, const int32_t *block_table,
+                       int max_pages, const int32_t *kv_len, const int32_t *markers,
+                       const int32_t *q_offsets, int R, int T_cap, int Hq, int Hkv, int D,
+                       int K, int page_size, int dtype, float scale, void *out,
+                       void *ws, size_t ws_bytes, dspark_stream_t stream);
+
+/* Workspace of dspark_accept: per-row softmax statistics. */
+size_t dspark_accept_workspace_bytes(int R, int K, int T_cap);
+
+/*
+ * dspark_accept — exact acceptance, longest accepted prefix, correction / bonus token.
+ *
+ * Defined by [P2 §一] (verify the N draft tokens in one pass, keep the verified ones,
+ * resample after the first divergence; the output distribution equals the target's),
+ * [P3 "DSpark的神奇之处"] (from the first wrong guess the large model writes a correct token
+ * itself) and [P3 "成本与质量的考量"] (the acceptance rule preserves the target distribution
+ * exactly).  With p_j = softmax(target row q_offsets[r]+j / temperature) and
+ * q_j = softmax(draft_logits[r][j] / temperature):
+ *   draft token k (k = 0..L-1, L = verify_len[r]) is accepted iff
+ *       u_acc[r][k] < min(1, p_k(x_k) / q_k(x_k));
+ *   a = accepted count before the first rejection;
+ *   a < L : correction drawn from max(0, p_a - q_a) (normalised), a == L: bonus from p_L;
+ *   draw = smallest v with C(v) > u_res[r][a] * C(V-1), C the running sum in index order.
+ * temperature <= 0 selects greedy verification: accept iff x_k == argmax of target row k
+ * (lowest index on ties); the correction / bonus is the argmax of target row a.
+ *
+ * target_logits [T_cap][V] (row q_offsets[r] + j = position j+1 of request r),
+ * draft_logits [R][K][V], dtype DSPARK_BF16 or DSPARK_F32; draft_tokens int32 [R][K];
+ * verify_len int32 [R]; q_offsets int32 [R + 1]; u_acc float32 [R][K]; u_res float32
+ * [R][K + 1] (uniforms in [0, 1)).  Outputs: accepted_len int32 [R]; out_tokens int32
+ * [R][K + 1] (accepted drafts, then the correction / bonus, then -1); n_out int32 [R] = a + 1.
+ * In greedy mode draft_logits, u_acc and u_res may be NULL.
+ */
+int dspark_accept(const void *target_logits, const void *draft_logits, int dtype, int V,
+                  int R, int K, int T_cap, const int32_t *draft_tokens,
+                  const int32_t *verify_len, const int32_t *q_offsets, const float *u_acc,
+                  const float *u_res, float temperature, int32_t *accepted_len,
+                  int32_t *out_tokens, int32_t *n_out, void *ws, size_t ws_bytes,
+                  dspark_stream_t stream);
+
+/*
+ * dspark_read_error — synchronise `stream`, return the current device's sticky error word
+ * in *host_code (HOST pointer; 0 = no error, else DSPARK_DERR_* bits) and clear it.
+ * Returns DSPARK_OK, or DSPARK_ECUDA if the synchronisation or copy failed.
+ */
+int dspark_read_error(int32_t *host_code, dspark_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSPARK_H */

@@ -1,0 +1,138 @@
+// Work partition and split-KV merge shared by the verify-attention kernels.
+//
+// The flattened verify batch ("刚融完500亿…专治AI“嘴慢”", engineering table row "内核利用率暴跌":
+// every verify token is an independent element, no per-request padding) is turned into a
+// sequence of work units: for each request r (in order) and each KV head g, the request's cache
+// is cut into tiles of kTileKeys positions (at least one tile, so that requests with an empty
+// cache still process their own verify tokens).  A segment = all tiles of one (r, g); all G*Q_r
+// query rows of the segment are processed together, so every KV byte is read once.
+//
+// The unit sequence is split into equal contiguous ranges, one per persistent CTA (W units
+// each).  A segment cut by a range boundary is computed in pieces; each piece writes an
+// un-normalised (m, l, acc) partial and the last piece to arrive (atomic counter, no waiting)
+// merges them.  CTA c writes at most two partials: slot 2c for its first segment, 2c+1 for its
+// last one.
+#pragma once
+
+#include "common.cuh"
+
+namespace dspark {
+
+constexpr int kTileKeys = 64;
+constexpr int kMaxCtasPerSm = 4;
+
+struct AttnPlanHeader {
+  int R, Hkv, rows_max, D;
+  int tile_keys, pad0, pad1, pad2;
+};
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct AttnWs {
+  AttnPlanHeader *hdr;
+  int *tile_prefix;  // [R + 1]: first unit of request r (units of all its Hkv segments)
+  int *counters;     // [R * Hkv] arrival counters of split segments (kept at zero between calls)
+  float *partials;   // [2 * max_ctas][rows_max][D + 2]: acc[D], m, l per row
+};
+
+__host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, int D,
+                                                 int max_ctas, AttnWs *ws, void *base) {
+  size_t off = 0;
+  const size_t o_hdr = off;                off += align256(sizeof(AttnPlanHeader));
+  const size_t o_pre = off;                off += align256((size_t)(R + 1) * sizeof(int));
+  const size_t o_cnt = off;                off += align256((size_t)R * Hkv * sizeof(int));
+  const size_t o_par = off;
+  off += align256((size_t)2 * max_ctas * rows_max * (D + 2) * sizeof(float));
+  if (ws) {
+    char *b = static_cast<char *>(base);
+    ws->hdr = reinterpret_cast<AttnPlanHeader *>(b + o_hdr);
+    ws->tile_prefix = reinterpret_cast<int *>(b + o_pre);
+    ws->counters = reinterpret_cast<int *>(b + o_cnt);
+    ws->partials = reinterpret_cast<float *>(b + o_par);
+  }
+  return off;
+}
+
+// Plan: tile_prefix (exclusive scan of Hkv * max(1, ceil(kv_len / kTileKeys))) and counters = 0.
+__global__ void __launch_bounds__(1024)
+attn_plan_kernel(const int32_t *__restrict__ kv_len, int R, int Hkv, int rows_max, int D,
+                 AttnWs ws) {
+  __shared__ int warp_tot[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (R + blockDim.x - 1) / blockDim.x;
+  int local = 0;
+  for (int i = 0; i < per; ++i) {
+    const int r = tid * per + i;
+    if (r < R) {
+      int n = kv_len[r];
+      if (n < 0) { raise_error(DSPARK_DERR_KV_LEN); n = 0; }
+      local += Hkv * max(1, (n + kTileKeys - 1) / kTileKeys);
+    }
+  }
+  int incl = local;
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int v = (lane < (int)(blockDim.x >> 5)) ? warp_tot[lane] : 0;
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    warp_tot[lane] = v;
+  }
+  __syncthreads();
+  int off = (warp ? warp_tot[warp - 1] : 0) + incl - local;
+  for (int i = 0; i < per; ++i) {
+    const int r = tid * per + i;
+    if (r < R) {
+      ws.tile_prefix[r] = off;
+      int n = max(kv_len[r], 0);
+      off += Hkv * max(1, (n + kTileKeys - 1) / kTileKeys);
+      if (r == R - 1) ws.tile_prefix[R] = off;
+    }
+  }
+  for (int i = tid; i < R * Hkv; i += blockDim.x) ws.counters[i] = 0;
+  if (tid == 0) {
+    ws.hdr->R = R;
+    ws.hdr->Hkv = Hkv;
+    ws.hdr->rows_max = rows_max;
+    ws.hdr->D = D;
+    ws.hdr->tile_keys = kTileKeys;
+  }
+}
+
+// A contiguous piece of one segment handled by one CTA.
+struct SegPiece {
+  int r, g;         // request, KV head
+  int ta, tb;       // tile range [ta, tb) within the segment
+  int tiles;        // tiles in the whole segment
+  int seg_start;    // global index of the segment's first unit
+  bool first_of_cta;
+};
+
+// Locate the segment containing global unit u (binary search over requests).
+__device__ __forceinline__ void find_segment(const int *__restrict__ tile_prefix, int R, int Hkv,
+                                             int u, int &r, int &g, int &tiles, int &seg_start) {
+  int lo = 0, hi = R - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(tile_prefix + mid) <= u) lo = mid; else hi = mid - 1;
+  }
+  r = lo;
+  const int base = __ldg(tile_prefix + r);
+  tiles = (__ldg(tile_prefix + r + 1) - base) / Hkv;
+  g = (u - base) / tiles;
+  seg_start = base + g * tiles;
+}
+
+// Slot of the partial written for segment (start s0, tiles nt) by CTA c, given W units per CTA.
+__device__ __forceinline__ int partial_slot(int c, int s0, int W) {
+  const int first_cta = s0 / W;
+  return 2 * c + ((c == first_cta && s0 != c * W) ? 1 : 0);
+}
+
+}  // namespace dspark

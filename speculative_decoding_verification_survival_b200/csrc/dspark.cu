@@ -1,0 +1,231 @@
+// libdspark: C ABI entry points (include/dspark.h).  Host-side validation, launch shapes and
+// dispatch; the kernels live in the included headers so that the whole library is one module
+// with one device error word.
+#include <cmath>
+#include <cstdio>
+
+#include "common.cuh"
+#include "schedule.cuh"
+#include "attn_common.cuh"
+#include "attn_generic.cuh"
+#include "accept.cuh"
+
+using namespace dspark;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return n;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DSPARK_OK : DSPARK_ECUDA;
+}
+
+int max_attn_ctas() {
+  const int sms = sm_count();
+  return sms > 0 ? sms * kMaxCtasPerSm : -1;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *dspark_status_string(int status) {
+  switch (status) {
+    case DSPARK_OK: return "DSPARK_OK";
+    case DSPARK_EINVAL: return "DSPARK_EINVAL: invalid argument";
+    case DSPARK_ECUDA: return "DSPARK_ECUDA: CUDA runtime error";
+    case DSPARK_EWORKSPACE: return "DSPARK_EWORKSPACE: workspace missing or too small";
+    case DSPARK_EDEVICE_DATA: return "DSPARK_EDEVICE_DATA: invalid device-resident data";
+    case DSPARK_ETIMEOUT: return "DSPARK_ETIMEOUT: bounded wait expired";
+    case DSPARK_EUNSUPPORTED: return "DSPARK_EUNSUPPORTED: shape not supported by this build";
+    default: return "DSPARK_UNKNOWN_STATUS";
+  }
+}
+
+int dspark_version(void) { return kVersion; }
+
+int dspark_schedule(const float *conf_ring, int ring_depth, int round_idx, int R, int K,
+                    const int32_t *kv_len, const double *t_ms, int T_cap, int32_t *verify_len,
+                    int32_t *q_offsets, int32_t *markers, int32_t *T_out, double *objective,
+                    dspark_stream_t stream) {
+  if (!conf_ring || !kv_len || !t_ms || !verify_len || !q_offsets || !markers || !T_out ||
+      !objective)
+    return DSPARK_EINVAL;
+  if (R < 1 || K < 1 || K > DSPARK_MAX_K || ring_depth < DSPARK_CONF_LAG + 1 || round_idx < 0 ||
+      T_cap < R)
+    return DSPARK_EINVAL;
+  if ((int64_t)R * K > DSPARK_MAX_CANDIDATES) return DSPARK_EUNSUPPORTED;
+  const int N = R * K;
+  int E = 1;
+  while (kSchedThreads * E < N) E *= 2;
+  const size_t smem = schedule_smem_bytes(E);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+#define DSPARK_SCHED_LAUNCH(EE)                                                                \
+  do {                                                                                         \
+    if (cudaFuncSetAttribute(schedule_kernel<EE>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             (int)smem) != cudaSuccess)                                        \
+      return DSPARK_ECUDA;                                                                     \
+    schedule_kernel<EE><<<1, kSchedThreads, smem, s>>>(conf_ring, ring_depth, round_idx, R, K, \
+                                                       kv_len, t_ms, T_cap, verify_len,        \
+                                                       q_offsets, markers, T_out, objective);  \
+  } while (0)
+  switch (E) {
+    case 1: DSPARK_SCHED_LAUNCH(1); break;
+    case 2: DSPARK_SCHED_LAUNCH(2); break;
+    case 4: DSPARK_SCHED_LAUNCH(4); break;
+    case 8: DSPARK_SCHED_LAUNCH(8); break;
+    case 16: DSPARK_SCHED_LAUNCH(16); break;
+    default: return DSPARK_EUNSUPPORTED;
+  }
+#undef DSPARK_SCHED_LAUNCH
+  return launch_status();
+}
+
+size_t dspark_verify_attn_workspace_bytes(int R, int Hq, int Hkv, int D, int K) {
+  if (R < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || D < 1 || K < 1 || K > DSPARK_MAX_K)
+    return 0;
+  const int ctas = max_attn_ctas();
+  if (ctas <= 0) return 0;
+  return attn_ws_layout(R, Hkv, (Hq / Hkv) * (K + 1), D, ctas, nullptr, nullptr);
+}
+
+int dspark_verify_attn_plan(const int32_t *kv_len, int R, int Hq, int Hkv, int D, int K, void *ws,
+                            size_t ws_bytes, dspark_stream_t stream) {
+  if (!kv_len || R < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || D < 8 || D > 256 || D % 8 ||
+      K < 1 || K > DSPARK_MAX_K)
+    return DSPARK_EINVAL;
+  if (!ws || !aligned16(ws)) return DSPARK_EWORKSPACE;
+  const int ctas = max_attn_ctas();
+  if (ctas <= 0) return DSPARK_ECUDA;
+  const int rows_max = (Hq / Hkv) * (K + 1);
+  AttnWs w;
+  if (ws_bytes < attn_ws_layout(R, Hkv, rows_max, D, ctas, &w, ws)) return DSPARK_EWORKSPACE;
+  attn_plan_kernel<<<1, 1024, 0, reinterpret_cast<cudaStream_t>(stream)>>>(kv_len, R, Hkv,
+                                                                           rows_max, D, w);
+  return launch_status();
+}
+
+int dspark_verify_attn(const void *q, const void *k_new, const void *v_new, const void *kv_pages,
+                       int64_t num_pages, const int32_t *block_table, int max_pages,
+                       const int32_t *kv_len, const int32_t *markers, const int32_t *q_offsets,
+                       int R, int T_cap, int Hq, int Hkv, int D, int K, int page_size, int dtype,
+                       float scale, void *out, void *ws, size_t ws_bytes,
+                       dspark_stream_t stream) {
+  if (!q || !k_new || !v_new || !kv_pages || !block_table || !kv_len || !markers || !q_offsets ||
+      !out)
+    return DSPARK_EINVAL;
+  if (R < 1 || T_cap < R || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || K < 1 || K > DSPARK_MAX_K ||
+      page_size < 1 || max_pages < 1 || num_pages < 1 || !std::isfinite(scale))
+    return DSPARK_EINVAL;
+  if (D < 8 || D > 256 || D % 8 != 0) return DSPARK_EUNSUPPORTED;
+  if (dtype != DSPARK_BF16 && dtype != DSPARK_F32) return DSPARK_EINVAL;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(kv_pages) ||
+      !aligned16(out))
+    return DSPARK_EINVAL;
+  const int G = Hq / Hkv;
+  const int rows_max = G * (K + 1);
+  if (rows_max > 128) return DSPARK_EUNSUPPORTED;
+  if (!ws || !aligned16(ws)) return DSPARK_EWORKSPACE;
+  const int sms = sm_count();
+  if (sms <= 0) return DSPARK_ECUDA;
+  AttnWs w;
+  if (ws_bytes < attn_ws_layout(R, Hkv, rows_max, D, sms * kMaxCtasPerSm, &w, ws))
+    return DSPARK_EWORKSPACE;
+
+  AttnArgs a;
+  a.q = q; a.k_new = k_new; a.v_new = v_new; a.kv_pages = kv_pages; a.num_pages = num_pages;
+  a.block_table = block_table; a.max_pages = max_pages; a.kv_len = kv_len; a.markers = markers;
+  a.q_offsets = q_offsets; a.R = R; a.T_cap = T_cap; a.Hq = Hq; a.Hkv = Hkv; a.G = G; a.D = D;
+  a.K = K; a.page_size = page_size; a.rows_max = rows_max;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.out = out; a.ws = w;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t smem = attn_generic_smem_bytes(rows_max, D);
+  if (smem > 227 * 1024) return DSPARK_EUNSUPPORTED;
+  auto launch = [&](auto kernel) -> int {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return DSPARK_ECUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kGenThreads, smem) !=
+        cudaSuccess)
+      return DSPARK_ECUDA;
+    per_sm = std::max(1, std::min(per_sm, kMaxCtasPerSm));
+    kernel<<<sms * per_sm, kGenThreads, smem, s>>>(a);
+    return launch_status();
+  };
+  if (dtype == DSPARK_BF16) return launch(attn_generic_kernel<__nv_bfloat16>);
+  return launch(attn_generic_kernel<float>);
+}
+
+size_t dspark_accept_workspace_bytes(int R, int K, int T_cap) {
+  if (R < 1 || K < 1 || K > DSPARK_MAX_K || T_cap < R) return 0;
+  return accept_ws_bytes(R, K, T_cap);
+}
+
+int dspark_accept(const void *target_logits, const void *draft_logits, int dtype, int V, int R,
+                  int K, int T_cap, const int32_t *draft_tokens, const int32_t *verify_len,
+                  const int32_t *q_offsets, const float *u_acc, const float *u_res,
+                  float temperature, int32_t *accepted_len, int32_t *out_tokens, int32_t *n_out,
+                  void *ws, size_t ws_bytes, dspark_stream_t stream) {
+  const bool greedy = !(temperature > 0.f);
+  if (!target_logits || !draft_tokens || !verify_len || !q_offsets || !accepted_len ||
+      !out_tokens || !n_out)
+    return DSPARK_EINVAL;
+  if (!greedy && (!draft_logits || !u_acc || !u_res)) return DSPARK_EINVAL;
+  if (std::isnan(temperature) || std::isinf(temperature)) return DSPARK_EINVAL;
+  if (V < 1 || R < 1 || K < 1 || K > DSPARK_MAX_K || T_cap < R) return DSPARK_EINVAL;
+  if (dtype != DSPARK_BF16 && dtype != DSPARK_F32) return DSPARK_EINVAL;
+  if (!ws || ws_bytes < accept_ws_bytes(R, K, T_cap) || !aligned16(ws)) return DSPARK_EWORKSPACE;
+  const float c = greedy ? 0.f : (float)(1.4426950408889634 / (double)temperature);
+  RowStats *st = static_cast<RowStats *>(ws);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int nrows = T_cap + R * K;
+  const int nch = (V + kAccChunk - 1) / kAccChunk;
+  const size_t fin_smem = (size_t)(nch + 2) * sizeof(double);
+  if (fin_smem > 227 * 1024) return DSPARK_EUNSUPPORTED;
+  auto run = [&](auto tag) -> int {
+    using T = decltype(tag);
+    const T *tl = static_cast<const T *>(target_logits);
+    const T *dl = static_cast<const T *>(draft_logits);
+    accept_stats_kernel<T><<<nrows, kAccThreads, 0, s>>>(tl, dl, V, R, K, T_cap, verify_len,
+                                                         q_offsets, c, greedy ? 1 : 0, st);
+    if (cudaGetLastError() != cudaSuccess) return DSPARK_ECUDA;
+    if (fin_smem > 48 * 1024 &&
+        cudaFuncSetAttribute(accept_finalize_kernel<T>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)fin_smem) != cudaSuccess)
+      return DSPARK_ECUDA;
+    accept_finalize_kernel<T><<<R, kAccThreads, fin_smem, s>>>(
+        tl, dl, V, R, K, T_cap, draft_tokens, verify_len, q_offsets, u_acc, u_res, c,
+        greedy ? 1 : 0, st, accepted_len, out_tokens, n_out);
+    return launch_status();
+  };
+  if (dtype == DSPARK_BF16) return run(__nv_bfloat16());
+  return run(float());
+}
+
+int dspark_read_error(int32_t *host_code, dspark_stream_t stream) {
+  if (!host_code) return DSPARK_EINVAL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DSPARK_ECUDA;
+  if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof(int)) != cudaSuccess) return DSPARK_ECUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return DSPARK_ECUDA;
+  *host_code = v;
+  return DSPARK_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,181 @@
+"""Thin ctypes binding of libdspark (include/dspark.h): argument marshalling only.
+
+Every function below has the name of the C entry point it calls and forwards device pointers
+of caller-provided torch tensors plus the current CUDA stream.  Nothing here computes any part
+of the verify step; if the shared library is missing the import fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .build import LIB_PATH
+
+DSPARK_OK = 0
+DSPARK_F32 = 0
+DSPARK_BF16 = 1
+DSPARK_CONF_LAG = 2
+DSPARK_MAX_K = 16
+DSPARK_MAX_CANDIDATES = 16384
+
+DEVICE_ERROR_BITS = {
+    1 << 0: "CONF", 1 << 1: "TABLE", 1 << 2: "KV_LEN", 1 << 3: "PAGE", 1 << 4: "MARKER",
+    1 << 5: "OFFSETS", 1 << 6: "VERIFY_LEN", 1 << 7: "TOKEN", 1 << 8: "LOGITS",
+}
+
+
+class DSparkError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = _lib.dspark_status_string(status).decode() if _lib is not None else str(status)
+        super().__init__(f"{fn} failed: {msg} ({status})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libdspark.so is not built ({LIB_PATH}); run "
+                          "speculative_decoding_verification_survival_b200.build.build()")
+    return ctypes.CDLL(LIB_PATH)
+
+
+_lib = _load()
+_p = ctypes.c_void_p
+_i = ctypes.c_int
+_i64 = ctypes.c_int64
+_f = ctypes.c_float
+_sz = ctypes.c_size_t
+
+_SIGS = {
+    "dspark_status_string": ([_i], ctypes.c_char_p),
+    "dspark_version": ([], _i),
+    "dspark_schedule": ([_p, _i, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p], _i),
+    "dspark_verify_attn_workspace_bytes": ([_i, _i, _i, _i, _i], _sz),
+    "dspark_verify_attn_plan": ([_p, _i, _i, _i, _i, _i, _p, _sz, _p], _i),
+    "dspark_verify_attn": ([_p, _p, _p, _p, _i64, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i,
+                            _i, _i, _f, _p, _p, _sz, _p], _i),
+    "dspark_accept_workspace_bytes": ([_i, _i, _i], _sz),
+    "dspark_accept": ([_p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _f, _p, _p, _p, _p, _sz,
+                       _p], _i),
+    "dspark_read_error": ([ctypes.POINTER(ctypes.c_int32), _p], _i),
+}
+for _name, (_args, _ret) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _ret
+
+EXPORTED = tuple(_SIGS)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError("tensors passed to libdspark must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libdspark must be contiguous")
+    return t.data_ptr()
+
+
+def _check(t, dtype, name):
+    if t is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _call(name, *args):
+    st = getattr(_lib, name)(*args)
+    if st != DSPARK_OK:
+        raise DSparkError(name, st)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DSPARK_BF16
+    if t.dtype == torch.float32:
+        return DSPARK_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def dspark_version() -> int:
+    return _lib.dspark_version()
+
+
+def dspark_status_string(status: int) -> str:
+    return _lib.dspark_status_string(status).decode()
+
+
+def dspark_schedule(conf_ring, round_idx, kv_len, t_ms, T_cap, verify_len, q_offsets, markers,
+                    T_out, objective, stream=None):
+    """conf_ring float32 [depth][R][K]; kv_len int32 [R]; t_ms float64 [T_cap+1];
+    outputs verify_len int32 [R], q_offsets int32 [R+1], markers int32 [T_cap][2],
+    T_out int32 [1], objective float64 [1]."""
+    depth, R, K = conf_ring.shape
+    _check(conf_ring, torch.float32, "conf_ring")
+    _check(kv_len, torch.int32, "kv_len")
+    _check(t_ms, torch.float64, "t_ms")
+    _call("dspark_schedule", _ptr(conf_ring), depth, int(round_idx), R, K, _ptr(kv_len),
+          _ptr(t_ms), int(T_cap), _ptr(verify_len), _ptr(q_offsets), _ptr(markers), _ptr(T_out),
+          _ptr(objective), _stream(stream))
+
+
+def dspark_verify_attn_workspace_bytes(R, Hq, Hkv, D, K) -> int:
+    return int(_lib.dspark_verify_attn_workspace_bytes(R, Hq, Hkv, D, K))
+
+
+def dspark_verify_attn_plan(kv_len, R, Hq, Hkv, D, K, ws, stream=None):
+    _check(kv_len, torch.int32, "kv_len")
+    _call("dspark_verify_attn_plan", _ptr(kv_len), R, Hq, Hkv, D, K, _ptr(ws), ws.numel(),
+          _stream(stream))
+
+
+def dspark_verify_attn(q, k_new, v_new, kv_pages, block_table, kv_len, markers, q_offsets, K,
+                       scale, out, ws, stream=None):
+    """q [T_cap][Hq][D]; k_new/v_new [T_cap][Hkv][D]; kv_pages [P][2][Hkv][page][D];
+    block_table int32 [R][max_pages]; out [T_cap][Hq][D]."""
+    T_cap, Hq, D = q.shape
+    Hkv = k_new.shape[1]
+    num_pages, _, _, page_size, _ = kv_pages.shape
+    R, max_pages = block_table.shape
+    for t in (k_new, v_new, kv_pages, out):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k_new, v_new, kv_pages and out must share a dtype")
+    _call("dspark_verify_attn", _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(kv_pages), num_pages,
+          _ptr(block_table), max_pages, _ptr(kv_len), _ptr(markers), _ptr(q_offsets), R, T_cap,
+          Hq, Hkv, D, int(K), page_size, _dtype_code(q), float(scale), _ptr(out), _ptr(ws),
+          ws.numel(), _stream(stream))
+
+
+def dspark_accept_workspace_bytes(R, K, T_cap) -> int:
+    return int(_lib.dspark_accept_workspace_bytes(R, K, T_cap))
+
+
+def dspark_accept(target_logits, draft_logits, draft_tokens, verify_len, q_offsets, u_acc, u_res,
+                  temperature, accepted_len, out_tokens, n_out, ws, stream=None):
+    """target_logits [T_cap][V]; draft_logits [R][K][V] (None allowed when greedy);
+    draft_tokens int32 [R][K]; u_acc float32 [R][K]; u_res float32 [R][K+1]."""
+    T_cap, V = target_logits.shape
+    R, K = draft_tokens.shape
+    if draft_logits is not None and draft_logits.dtype != target_logits.dtype:
+        raise TypeError("target and draft logits must share a dtype")
+    _call("dspark_accept", _ptr(target_logits), _ptr(draft_logits), _dtype_code(target_logits),
+          V, R, K, T_cap, _ptr(draft_tokens), _ptr(verify_len), _ptr(q_offsets), _ptr(u_acc),
+          _ptr(u_res), float(temperature), _ptr(accepted_len), _ptr(out_tokens), _ptr(n_out),
+          _ptr(ws), ws.numel(), _stream(stream))
+
+
+def dspark_read_error(stream=None) -> int:
+    code = ctypes.c_int32(0)
+    _call("dspark_read_error", ctypes.byref(code), _stream(stream))
+    return int(code.value)
+
+
+def decode_device_error(code: int):
+    return [name for bit, name in DEVICE_ERROR_BITS.items() if code & bit]

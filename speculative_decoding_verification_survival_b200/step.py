@@ -1,0 +1,69 @@
+"""One confidence-scheduled verify step on one GPU, composed from the libdspark entry points.
+
+    schedule (lagged confidences -> verify lengths, offsets, markers)
+      -> attention plan (work partition of the step, reused by every layer)
+      -> one flattened verify-attention call per layer
+      -> accept (acceptance test, longest prefix, correction / bonus token)
+
+VerifyStep owns the step's device outputs and workspaces (allocated once through torch) and
+issues the calls in order on the current stream.  It does no arithmetic of its own.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import dspark as _d
+
+
+class VerifyStep:
+    def __init__(self, R: int, K: int, Hq: int, Hkv: int, D: int, V: int, device="cuda",
+                 T_cap: int | None = None):
+        self.R, self.K, self.Hq, self.Hkv, self.D, self.V = R, K, Hq, Hkv, D, V
+        self.T_cap = R * (K + 1) if T_cap is None else T_cap
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.verify_len = torch.zeros(R, **i32)
+        self.q_offsets = torch.zeros(R + 1, **i32)
+        self.markers = torch.zeros(self.T_cap, 2, **i32)
+        self.T = torch.zeros(1, **i32)
+        self.objective = torch.zeros(1, dtype=torch.float64, device=dev)
+        self.accepted_len = torch.zeros(R, **i32)
+        self.out_tokens = torch.zeros(R, K + 1, **i32)
+        self.n_out = torch.zeros(R, **i32)
+        nbytes = _d.dspark_verify_attn_workspace_bytes(R, Hq, Hkv, D, K)
+        self.attn_ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=dev)
+        nbytes = _d.dspark_accept_workspace_bytes(R, K, self.T_cap)
+        self.accept_ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=dev)
+        self.scale = 1.0 / math.sqrt(D)
+
+    def schedule(self, conf_ring, round_idx, kv_len, t_ms, stream=None):
+        _d.dspark_schedule(conf_ring, round_idx, kv_len, t_ms, self.T_cap, self.verify_len,
+                           self.q_offsets, self.markers, self.T, self.objective, stream)
+
+    def plan(self, kv_len, stream=None):
+        _d.dspark_verify_attn_plan(kv_len, self.R, self.Hq, self.Hkv, self.D, self.K,
+                                   self.attn_ws, stream)
+
+    def attention(self, q, k_new, v_new, kv_pages, block_table, kv_len, out, stream=None):
+        _d.dspark_verify_attn(q, k_new, v_new, kv_pages, block_table, kv_len, self.markers,
+                              self.q_offsets, self.K, self.scale, out, self.attn_ws, stream)
+
+    def accept(self, target_logits, draft_logits, draft_tokens, u_acc, u_res, temperature,
+               stream=None):
+        _d.dspark_accept(target_logits, draft_logits, draft_tokens, self.verify_len,
+                         self.q_offsets, u_acc, u_res, temperature, self.accepted_len,
+                         self.out_tokens, self.n_out, self.accept_ws, stream)
+
+    def run(self, conf_ring, round_idx, kv_len, t_ms, layers, kv_pages_per_layer, block_table,
+            attn_out, target_logits, draft_logits, draft_tokens, u_acc, u_res, temperature,
+            stream=None) -> int:
+        """Issue one whole step; `layers` is a sequence of (q, k_new, v_new) per layer and
+        kv_pages_per_layer the matching caches.  Returns the number of kernels launched."""
+        self.schedule(conf_ring, round_idx, kv_len, t_ms, stream)
+        self.plan(kv_len, stream)
+        for (q, k_new, v_new), kv in zip(layers, kv_pages_per_layer):
+            self.attention(q, k_new, v_new, kv, block_table, kv_len, attn_out, stream)
+        self.accept(target_logits, draft_logits, draft_tokens, u_acc, u_res, temperature, stream)
+        return 2 + len(layers) + 2

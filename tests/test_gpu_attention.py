@@ -1,0 +1,156 @@
+"""GPU verify-attention parity against the float64 oracle on identical bf16 / f32 inputs.
+
+Small cases compare every output element (several 64-key tiles, ragged tails, empty caches,
+zero-length schedules, page crossings, all GQA group sizes used by the workloads); the full
+workloads compare sampled (token, head) rows computed one by one by the oracle.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.gpu_support import (ATTN_MAX_ABS, ATTN_MEAN_ABS, F32_ATTN_MAX_ABS, binding, host,
+                               new_step, oracle_attn_rows, set_schedule)
+from workloads.configs import CONFIGS, TINY, QWEN3_4B
+from workloads.generate import build_step_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_attn(step, inp, layer=0, cache=None):
+    cache = inp.kv_caches[0] if cache is None else cache
+    out = torch.full_like(inp.q[layer], float("nan"))
+    step.plan(inp.kv_len)
+    step.attention(inp.q[layer], inp.k_new[layer], inp.v_new[layer], cache, inp.block_table,
+                   inp.kv_len, out)
+    torch.cuda.synchronize()
+    return out
+
+
+def _full_compare(cfg, verify_len, seed=0, tol=None):
+    inp = build_step_inputs(cfg, "cuda", seed=seed, layers=1)
+    step = new_step(cfg)
+    kv = host(inp.kv_len)
+    qo, mk = set_schedule(step, verify_len, kv)
+    out = _run_attn(step, inp)
+    T = int(qo[-1])
+    ref = oracle.attn_ref_flat(host(inp.q[0, :T]), host(inp.k_new[0, :T]), host(inp.v_new[0, :T]),
+                               host(inp.kv_caches[0]), host(inp.block_table), kv, mk, qo,
+                               step.scale, cfg.page_size)
+    got = host(out[:T]).astype(np.float64)
+    err = np.abs(got - ref)
+    assert np.all(np.isfinite(got))
+    if cfg.dtype == "f32":
+        assert err.max() <= (tol or F32_ATTN_MAX_ABS), err.max()
+    else:
+        assert err.max() <= ATTN_MAX_ABS and err.mean() <= ATTN_MEAN_ABS, (err.max(), err.mean())
+    assert binding().dspark_read_error() == 0
+    return err
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_tiny_f32_all_rows(seed):
+    rng = np.random.default_rng(seed)
+    L = rng.integers(0, TINY.K + 1, size=TINY.R)
+    _full_compare(TINY, L, seed=seed)
+
+
+@pytest.mark.parametrize("G,R,lo,hi", [(4, 6, 0, 300), (5, 5, 60, 200), (8, 4, 1, 129),
+                                       (8, 3, 0, 0)])
+def test_bf16_all_rows_several_tiles(G, R, lo, hi):
+    cfg = QWEN3_4B.with_(R=R, Hq=2 * G, Hkv=2, kv_dist=("uniform", lo, hi), V=64)
+    rng = np.random.default_rng(G * 100 + R)
+    L = rng.integers(0, cfg.K + 1, size=R)
+    L[0] = 0
+    L[-1] = cfg.K
+    _full_compare(cfg, L, seed=G)
+
+
+def test_bf16_small_pages_and_f32_head_dim_64():
+    cfg = QWEN3_4B.with_(R=5, Hq=8, Hkv=2, page_size=16, kv_dist=("uniform", 1, 150), V=64)
+    _full_compare(cfg, [5, 0, 3, 1, 2], seed=3)
+    cfg = TINY.with_(R=3, Hq=6, Hkv=3, D=64, page_size=32, kv_dist=("uniform", 40, 140))
+    _full_compare(cfg, [2, 5, 0], seed=4)
+
+
+def test_f32_long_cache_many_split_pieces():
+    # one request much longer than the rest: its segments are cut across many CTAs
+    cfg = TINY.with_(R=3, kv_dist=("uniform", 5000, 5000), D=32, page_size=8)
+    _full_compare(cfg, [5, 5, 5], seed=5)
+
+
+@pytest.mark.parametrize("name", ["qwen3-4b-64req", "mixed-256req", "lognormal-1024req",
+                                  "sweep-1req", "sweep-2048req"])
+def test_full_workload_sampled_rows(name):
+    cfg = CONFIGS[name]
+    inp = build_step_inputs(cfg, "cuda", seed=0, layers=1)
+    step = new_step(cfg)
+    step.schedule(inp.conf_ring, inp.round_idx, inp.kv_len, inp.t_ms)
+    out = _run_attn(step, inp)
+    T = int(step.T.item())
+    qo = host(step.q_offsets)
+    mk = host(step.markers)[:T]
+    rng = np.random.default_rng(1)
+    toks = set(rng.integers(0, T, size=40).tolist()) | {0, T - 1}
+    # include the longest request's tokens and a zero-length request if any
+    kv = host(inp.kv_len)
+    r_long = int(np.argmax(kv))
+    toks |= {int(qo[r_long]), int(qo[r_long + 1]) - 1}
+    rows = [(t, int(rng.integers(0, cfg.Hq))) for t in sorted(toks)]
+    ref = oracle_attn_rows(inp, 0, inp.kv_caches[0], qo, mk, rows, step.scale)
+    errs = np.concatenate([np.abs(host(out[t, h]).astype(np.float64) - ref[(t, h)])
+                           for t, h in rows])
+    assert errs.max() <= ATTN_MAX_ABS and errs.mean() <= ATTN_MEAN_ABS, (errs.max(), errs.mean())
+    # rows past the scheduled total are never written
+    if T < cfg.T_cap:
+        assert torch.isnan(out[T:]).all()
+    assert binding().dspark_read_error() == 0
+
+
+def test_repeated_calls_reuse_plan_and_counters():
+    cfg = QWEN3_4B.with_(R=7, kv_dist=("uniform", 100, 2000), V=64)
+    inp = build_step_inputs(cfg, "cuda", seed=9, layers=3)
+    step = new_step(cfg)
+    rng = np.random.default_rng(2)
+    qo, mk = set_schedule(step, rng.integers(0, 6, size=7), host(inp.kv_len))
+    step.plan(inp.kv_len)
+    outs = []
+    for layer in range(3):
+        out = torch.empty_like(inp.q[layer])
+        step.attention(inp.q[layer], inp.k_new[layer], inp.v_new[layer], inp.kv_caches[0],
+                       inp.block_table, inp.kv_len, out)
+        outs.append(out)
+    out0b = torch.empty_like(inp.q[0])
+    step.attention(inp.q[0], inp.k_new[0], inp.v_new[0], inp.kv_caches[0], inp.block_table,
+                   inp.kv_len, out0b)
+    torch.cuda.synchronize()
+    T = int(qo[-1])
+    assert torch.equal(outs[0][:T], out0b[:T])   # deterministic, counters reset
+    kv = host(inp.kv_len)
+    for layer in (1, 2):
+        ref = oracle.attn_ref_flat(host(inp.q[layer, :T]), host(inp.k_new[layer, :T]),
+                                   host(inp.v_new[layer, :T]), host(inp.kv_caches[0]),
+                                   host(inp.block_table), kv, mk, qo, step.scale, cfg.page_size)
+        err = np.abs(host(outs[layer][:T]) - ref)
+        assert err.max() <= ATTN_MAX_ABS and err.mean() <= ATTN_MEAN_ABS
+
+
+def test_corrupt_marker_and_page_set_error_bits():
+    d = binding()
+    cfg = QWEN3_4B.with_(R=4, kv_dist=("uniform", 10, 300), V=64)
+    inp = build_step_inputs(cfg, "cuda", seed=1, layers=1)
+    step = new_step(cfg)
+    set_schedule(step, [1, 2, 0, 3], host(inp.kv_len))
+    step.markers[1, 1] += 1            # wrong position for request 0's second token
+    _run_attn(step, inp)
+    assert d.dspark_read_error() & (1 << 4)
+    set_schedule(step, [1, 2, 0, 3], host(inp.kv_len))
+    bt = inp.block_table.clone()
+    bt[2, 0] = 10 ** 7                 # page outside the cache
+    out = torch.empty_like(inp.q[0])
+    step.plan(inp.kv_len)
+    step.attention(inp.q[0], inp.k_new[0], inp.v_new[0], inp.kv_caches[0], bt, inp.kv_len, out)
+    assert d.dspark_read_error() & (1 << 3)
+    assert d.dspark_read_error() == 0
