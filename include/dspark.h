@@ -205,6 +205,36 @@ int dspark_accept(const void *target_logits, const void *draft_logits, int dtype
                   dspark_stream_t stream);
 
 /*
+ * dspark_accept_noalloc — dspark_accept for callers that cannot allocate device memory.
+ *
+ * The paper has no counterpart to this entry point; it exists for library users.  Some hosts
+ * of this library may not call cudaMalloc: an inference engine whose memory pool has already
+ * reserved the GPU's free memory at start-up, a plugin running inside a runtime that forbids
+ * allocation after initialisation, or a latency-critical loop where an allocation (which can
+ * synchronise the device) is not acceptable.  They still pass their own inputs and outputs,
+ * but get the acceptance kernels' scratch (per-row softmax statistics) from a fixed array
+ * compiled into the library instead of a workspace argument.
+ *
+ * Arguments and results are those of dspark_accept without ws / ws_bytes.
+ * Limit: T_cap + R*K <= DSPARK_ACCEPT_NOALLOC_MAX_ROWS; larger calls return
+ * DSPARK_EUNSUPPORTED before anything is enqueued.  The array (16 bytes per row, 1 MiB) is held
+ * by every GPU that loads the library until the process exits.
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current; make that first call before any stream capture.
+ * All calls on a device share the one array and it keeps the previous call's contents (every
+ * row a call reads is written by that call first).  Calls whose executions overlap on the GPU
+ * — on different streams, or from different host threads — race on the array: serialise them.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define DSPARK_ACCEPT_NOALLOC_MAX_ROWS 65536
+int dspark_accept_noalloc(const void *target_logits, const void *draft_logits, int dtype, int V,
+                          int R, int K, int T_cap, const int32_t *draft_tokens,
+                          const int32_t *verify_len, const int32_t *q_offsets,
+                          const float *u_acc, const float *u_res, float temperature,
+                          int32_t *accepted_len, int32_t *out_tokens, int32_t *n_out,
+                          dspark_stream_t stream);
+
+/*
  * dspark_read_error — synchronise `stream`, return the current device's sticky error word
  * in *host_code (HOST pointer; 0 = no error, else DSPARK_DERR_* bits) and clear it.
  * Returns DSPARK_OK, or DSPARK_ECUDA if the synchronisation or copy failed.

@@ -1,6 +1,7 @@
 // libdspark: C ABI entry points (include/dspark.h).  Host-side validation, launch shapes and
 // dispatch; the kernels live in the included headers so that the whole library is one module
 // with one device error word.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 
@@ -229,3 +230,42 @@ int dspark_read_error(int32_t *host_code, dspark_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// No-allocation variant of dspark_accept.
+//
+// For callers that must not allocate device memory (their memory pool owns the GPU, their host
+// runtime forbids allocation after start-up, or an allocation's implicit synchronisation is not
+// acceptable).  The per-row statistics the acceptance kernels need live in this fixed array
+// instead of a caller workspace.  In host code `g_accept_noalloc_scratch` only names the
+// symbol; its device address is looked up once per device (with that device current) and that
+// address is what the kernels receive.
+static __device__ __align__(256) RowStats g_accept_noalloc_scratch[DSPARK_ACCEPT_NOALLOC_MAX_ROWS];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::atomic<void *> g_noalloc_scratch_addr[kNoAllocMaxDevices];
+}  // namespace
+
+extern "C" int dspark_accept_noalloc(const void *target_logits, const void *draft_logits,
+                                     int dtype, int V, int R, int K, int T_cap,
+                                     const int32_t *draft_tokens, const int32_t *verify_len,
+                                     const int32_t *q_offsets, const float *u_acc,
+                                     const float *u_res, float temperature,
+                                     int32_t *accepted_len, int32_t *out_tokens,
+                                     int32_t *n_out, dspark_stream_t stream) {
+  if (R < 1 || K < 1 || K > DSPARK_MAX_K || T_cap < R) return DSPARK_EINVAL;
+  if ((int64_t)T_cap + (int64_t)R * K > DSPARK_ACCEPT_NOALLOC_MAX_ROWS) return DSPARK_EUNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSPARK_ECUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return DSPARK_EUNSUPPORTED;
+  void *scratch = g_noalloc_scratch_addr[dev].load(std::memory_order_acquire);
+  if (scratch == nullptr) {
+    if (cudaGetSymbolAddress(&scratch, g_accept_noalloc_scratch) != cudaSuccess || !scratch)
+      return DSPARK_ECUDA;
+    g_noalloc_scratch_addr[dev].store(scratch, std::memory_order_release);
+  }
+  return dspark_accept(target_logits, draft_logits, dtype, V, R, K, T_cap, draft_tokens,
+                       verify_len, q_offsets, u_acc, u_res, temperature, accepted_len,
+                       out_tokens, n_out, scratch, sizeof(g_accept_noalloc_scratch), stream);
+}

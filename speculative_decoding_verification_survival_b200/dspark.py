@@ -19,6 +19,7 @@ DSPARK_BF16 = 1
 DSPARK_CONF_LAG = 2
 DSPARK_MAX_K = 16
 DSPARK_MAX_CANDIDATES = 16384
+DSPARK_ACCEPT_NOALLOC_MAX_ROWS = 65536
 
 DEVICE_ERROR_BITS = {
     1 << 0: "CONF", 1 << 1: "TABLE", 1 << 2: "KV_LEN", 1 << 3: "PAGE", 1 << 4: "MARKER",
@@ -59,6 +60,8 @@ _SIGS = {
     "dspark_accept": ([_p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _f, _p, _p, _p, _p, _sz,
                        _p], _i),
     "dspark_read_error": ([ctypes.POINTER(ctypes.c_int32), _p], _i),
+    "dspark_accept_noalloc": ([_p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _f, _p, _p, _p,
+                               _p], _i),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -179,3 +182,17 @@ def dspark_read_error(stream=None) -> int:
 
 def decode_device_error(code: int):
     return [name for bit, name in DEVICE_ERROR_BITS.items() if code & bit]
+
+
+def dspark_accept_noalloc(target_logits, draft_logits, draft_tokens, verify_len, q_offsets, u_acc,
+                          u_res, temperature, accepted_len, out_tokens, n_out, stream=None):
+    """dspark_accept without a workspace argument, for callers that cannot allocate device
+    memory: the scratch is a fixed array inside the library (see include/dspark.h)."""
+    T_cap, V = target_logits.shape
+    R, K = draft_tokens.shape
+    if draft_logits is not None and draft_logits.dtype != target_logits.dtype:
+        raise TypeError("target and draft logits must share a dtype")
+    _call("dspark_accept_noalloc", _ptr(target_logits), _ptr(draft_logits),
+          _dtype_code(target_logits), V, R, K, T_cap, _ptr(draft_tokens), _ptr(verify_len),
+          _ptr(q_offsets), _ptr(u_acc), _ptr(u_res), float(temperature), _ptr(accepted_len),
+          _ptr(out_tokens), _ptr(n_out), _stream(stream))
