@@ -72,7 +72,8 @@ enum dspark_device_error {
   DSPARK_DERR_OFFSETS = 1 << 5,     /* q_offsets not a scan of 1 + verify_len within T_cap */
   DSPARK_DERR_VERIFY_LEN = 1 << 6,  /* verify_len outside [0, K] */
   DSPARK_DERR_TOKEN = 1 << 7,       /* a draft token outside [0, V) */
-  DSPARK_DERR_LOGITS = 1 << 8       /* a logit row whose maximum is not finite */
+  DSPARK_DERR_LOGITS = 1 << 8,      /* a logit row whose maximum is not finite */
+  DSPARK_DERR_TIMEOUT = 1 << 9      /* a bounded in-kernel wait expired; results undefined */
 };
 
 #define DSPARK_CONF_LAG 2             /* rounds between producing and consuming confidences */
@@ -159,8 +160,9 @@ int dspark_verify_attn_plan(const int32_t *kv_len, int R, int Hq, int Hkv, int D
  * kv_len     int32 [R]; markers int32 [T_cap][2]; q_offsets int32 [R + 1] (from the schedule;
  *            only rows t < q_offsets[R] are read or written).
  * out        [T_cap][Hq][D], same dtype as the inputs.
- * dtype      DSPARK_BF16 (tensor-core path when D == 128 and page_size % 64 == 0) or
- *            DSPARK_F32; scale is usually 1/sqrt(D).
+ * dtype      DSPARK_BF16 or DSPARK_F32; scale is usually 1/sqrt(D).  bf16 with D == 128,
+ *            page_size % 64 == 0 and the cache below 2^31 rows of D elements runs on the
+ *            tensor cores (tcgen05 + TMA); every other shape runs on CUDA cores.
  * Limits: 1 <= D <= 256 with D % 8 == 0, Hq % Hkv == 0, (Hq/Hkv)*(K+1) <= 128.
  */
 int dspark_verify_attn(const void *q, const void *k_new, const void *v_new,

@@ -24,6 +24,7 @@ DSPARK_ACCEPT_NOALLOC_MAX_ROWS = 65536
 DEVICE_ERROR_BITS = {
     1 << 0: "CONF", 1 << 1: "TABLE", 1 << 2: "KV_LEN", 1 << 3: "PAGE", 1 << 4: "MARKER",
     1 << 5: "OFFSETS", 1 << 6: "VERIFY_LEN", 1 << 7: "TOKEN", 1 << 8: "LOGITS",
+    1 << 9: "TIMEOUT",
 }
 
 

@@ -154,3 +154,57 @@ def test_corrupt_marker_and_page_set_error_bits():
     step.attention(inp.q[0], inp.k_new[0], inp.v_new[0], inp.kv_caches[0], bt, inp.kv_len, out)
     assert d.dspark_read_error() & (1 << 3)
     assert d.dspark_read_error() == 0
+
+
+def _compare_with_scale(cfg, verify_len, seed, scale, kv_transform=None):
+    inp = build_step_inputs(cfg, "cuda", seed=seed, layers=1)
+    if kv_transform is not None:
+        kv_transform(inp)
+    step = new_step(cfg)
+    kv = host(inp.kv_len)
+    qo, mk = set_schedule(step, verify_len, kv)
+    out = torch.full_like(inp.q[0], float("nan"))
+    d = binding()
+    step.plan(inp.kv_len)
+    d.dspark_verify_attn(inp.q[0], inp.k_new[0], inp.v_new[0], inp.kv_caches[0], inp.block_table,
+                         inp.kv_len, step.markers, step.q_offsets, cfg.K, scale, out, step.attn_ws)
+    torch.cuda.synchronize()
+    T = int(qo[-1])
+    ref = oracle.attn_ref_flat(host(inp.q[0, :T]), host(inp.k_new[0, :T]), host(inp.v_new[0, :T]),
+                               host(inp.kv_caches[0]), host(inp.block_table), kv, mk, qo, scale,
+                               cfg.page_size)
+    err = np.abs(host(out[:T]).astype(np.float64) - ref)
+    assert np.all(np.isfinite(host(out[:T])))
+    assert err.max() <= ATTN_MAX_ABS and err.mean() <= ATTN_MEAN_ABS, (err.max(), err.mean())
+    assert d.dspark_read_error() == 0
+
+
+@pytest.mark.parametrize("G", [4, 5, 8, 16])
+def test_tensor_core_path_group_sizes(G):
+    # bf16, D 128, page 64: the tcgen05 kernel; G*(K+1) spans the 4-, 2- and 1-copy layouts
+    cfg = QWEN3_4B.with_(R=6, Hq=2 * G, Hkv=2, kv_dist=("uniform", 1, 700), V=64)
+    L = np.array([5, 0, 3, 5, 1, 4])
+    _compare_with_scale(cfg, L, seed=G, scale=1.0 / math.sqrt(128))
+
+
+def test_tensor_core_rescale_path():
+    # scale 1 and keys that grow along the cache make the running maximum jump by far more than
+    # 2^8 from tile to tile, so O is rescaled in tensor memory
+    cfg = QWEN3_4B.with_(R=4, Hq=16, Hkv=2, kv_dist=("uniform", 300, 900), V=64)
+
+    def grow(inp):
+        P, _, Hkv, page, D = inp.kv_caches[0].shape
+        table = inp.block_table.cpu().numpy()
+        kvl = inp.kv_len.cpu().numpy()
+        for r in range(cfg.R):
+            for p in range(-(-int(kvl[r]) // page)):
+                pg = int(table[r, p])
+                f = 1.0 + 0.02 * p * page
+                inp.kv_caches[0][pg, 0] = (inp.kv_caches[0][pg, 0].float() * f).to(torch.bfloat16)
+
+    _compare_with_scale(cfg, np.array([5, 2, 0, 4]), seed=3, scale=1.0, kv_transform=grow)
+
+
+def test_tensor_core_pages_of_128():
+    cfg = QWEN3_4B.with_(R=5, page_size=128, kv_dist=("uniform", 1, 1000), V=64)
+    _compare_with_scale(cfg, np.array([5, 4, 3, 2, 1]), seed=6, scale=1.0 / math.sqrt(128))
