@@ -130,8 +130,9 @@ size_t dspark_verify_attn_workspace_bytes(int R, int Hq, int Hkv, int D, int K);
 /*
  * dspark_verify_attn_plan — partition one step's attention work across the GPU.
  *
- * Work is the sequence of (request r, KV head g, KV tile) units in request-major order, each
- * request contributing Hkv * max(1, ceil(kv_len[r] / 64)) units; the plan splits it into
+ * Work is the sequence of (request r, KV head g, unit) in request-major order, each request
+ * contributing Hkv * (ceil(kv_len[r] / 64) + 1) units (its 64-key cache tiles, then its own
+ * verify tokens); the plan splits it into
  * equal contiguous ranges, one per persistent CTA.  Call once per step after the schedule
  * (the partition depends only on kv_len and the request count), before any
  * dspark_verify_attn of that step; it also zeroes the workspace's arrival counters.
@@ -161,8 +162,9 @@ int dspark_verify_attn_plan(const int32_t *kv_len, int R, int Hq, int Hkv, int D
  *            only rows t < q_offsets[R] are read or written).
  * out        [T_cap][Hq][D], same dtype as the inputs.
  * dtype      DSPARK_BF16 or DSPARK_F32; scale is usually 1/sqrt(D).  bf16 with D == 128,
- *            page_size % 64 == 0 and the cache below 2^31 rows of D elements runs on the
- *            tensor cores (tcgen05 + TMA); every other shape runs on CUDA cores.
+ *            page_size % 64 == 0, K + 1 <= 16, (Hq/Hkv)*(K+1) <= 64 and the cache below 2^31
+ *            rows of D elements runs on the tensor cores (tcgen05 + TMA); every other shape
+ *            runs on CUDA cores.
  * Limits: 1 <= D <= 256 with D % 8 == 0, Hq % Hkv == 0, (Hq/Hkv)*(K+1) <= 128.
  */
 int dspark_verify_attn(const void *q, const void *k_new, const void *v_new,

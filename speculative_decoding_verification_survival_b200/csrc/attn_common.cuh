@@ -3,9 +3,10 @@
 // The flattened verify batch ("刚融完500亿…专治AI“嘴慢”", engineering table row "内核利用率暴跌":
 // every verify token is an independent element, no per-request padding) is turned into a
 // sequence of work units: for each request r (in order) and each KV head g, the request's cache
-// is cut into tiles of kTileKeys positions (at least one tile, so that requests with an empty
-// cache still process their own verify tokens).  A segment = all tiles of one (r, g); all G*Q_r
-// query rows of the segment are processed together, so every KV byte is read once.
+// is cut into tiles of kTileKeys positions, followed by one unit for the request's own verify
+// tokens (so a request with an empty cache still has one unit).  A segment = all units of one
+// (r, g); all G*Q_r query rows of the segment are processed together, so every KV byte is read
+// once.
 //
 // The unit sequence is split into equal contiguous ranges, one per persistent CTA (W units
 // each).  A segment cut by a range boundary is computed in pieces; each piece writes an
@@ -53,7 +54,10 @@ __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, i
   return off;
 }
 
-// Plan: tile_prefix (exclusive scan of Hkv * max(1, ceil(kv_len / kTileKeys))) and counters = 0.
+// Units of one (request, KV head) segment: cache tiles plus the verify-token unit.
+__host__ __device__ inline int segment_units(int n) { return (n + kTileKeys - 1) / kTileKeys + 1; }
+
+// Plan: tile_prefix (exclusive scan of Hkv * segment_units(kv_len)) and counters = 0.
 __global__ void __launch_bounds__(1024)
 attn_plan_kernel(const int32_t *__restrict__ kv_len, int R, int Hkv, int rows_max, int D,
                  AttnWs ws) {
@@ -66,7 +70,7 @@ attn_plan_kernel(const int32_t *__restrict__ kv_len, int R, int Hkv, int rows_ma
     if (r < R) {
       int n = kv_len[r];
       if (n < 0) { raise_error(DSPARK_DERR_KV_LEN); n = 0; }
-      local += Hkv * max(1, (n + kTileKeys - 1) / kTileKeys);
+      local += Hkv * segment_units(n);
     }
   }
   int incl = local;
@@ -91,7 +95,7 @@ attn_plan_kernel(const int32_t *__restrict__ kv_len, int R, int Hkv, int rows_ma
     if (r < R) {
       ws.tile_prefix[r] = off;
       int n = max(kv_len[r], 0);
-      off += Hkv * max(1, (n + kTileKeys - 1) / kTileKeys);
+      off += Hkv * segment_units(n);
       if (r == R - 1) ws.tile_prefix[R] = off;
     }
   }

@@ -158,7 +158,7 @@ attn_generic_kernel(AttnArgs a) {
     };
 
     if (rows > 0) {
-      for (int tile = ta; tile < tb; ++tile) {
+      for (int tile = ta; tile < min(tb, tiles - 1); ++tile) {  // cache tiles of this piece
         const int k0 = tile * kTileKeys, k1 = min(k0 + kTileKeys, n);
         for (int c0 = k0; c0 < k1; c0 += kGenKC) {
           const int nk = min(kGenKC, k1 - c0);
@@ -190,7 +190,7 @@ attn_generic_kernel(AttnArgs a) {
           chunk_update(nk, false);
         }
       }
-      if (tb == tiles) {  // the request's own verify tokens, causal by marker position
+      if (tb == tiles) {  // the segment's last unit: the request's own verify tokens, causal
         for (int idx = tid; idx < kGenKC * (D / 8); idx += kGenThreads) {
           const int kk = idx / (D / 8), d8 = idx % (D / 8);
           float kvv[8] = {0, 0, 0, 0, 0, 0, 0, 0}, vvv[8] = {0, 0, 0, 0, 0, 0, 0, 0};

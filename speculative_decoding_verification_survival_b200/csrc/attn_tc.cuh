@@ -1,27 +1,35 @@
-// Tensor-core verify attention for sm_100a (bf16, D = 128, page size a multiple of 64).
+// Tensor-core verify attention for sm_100a (bf16, D = 128, page size a multiple of 64,
+// K + 1 <= 16, G * (K + 1) <= 64).
 //
 // Same work partition and split-KV merge as the CUDA-core kernel (attn_common.cuh): a persistent
-// CTA per SM walks a contiguous range of (request, KV head, 64-key tile) units; every KV byte is
-// read once for all G*Q_r query rows of its (request, KV head) — the flattened, unpadded verify
-// batch of "刚融完500亿…专治AI“嘴慢”" (engineering table, row "内核利用率暴跌").
+// CTA per SM walks a contiguous range of (request, KV head, unit) work, the units of a segment
+// being its 64-key cache tiles followed by one unit for the request's own verify tokens; every
+// KV byte is read once for all G*Q_r query rows of its (request, KV head) — the flattened,
+// unpadded verify batch of "刚融完500亿…专治AI“嘴慢”" (engineering table, row "内核利用率暴跌").
+//
+// A tcgen05 MMA costs about the same time whatever its N (up to 256) on B200, so the kernel
+// minimises instructions per key: two 64-key pages form one 128-key tile, S = Q.K^T of a tile is
+// 8 MMAs (M 128, N 128, K 16) and O += P.V is 8 MMAs (M 128, N 128, K 16).
 //
 // Per CTA (192 threads):
-//   warp 4      TMA producer: per tile, one 64-row x 128-B box per d-half of the page's K and V
-//               tiles (128-byte swizzle) into a 4-stage shared-memory ring (32 KB per stage).
-//   warp 5      MMA issuer (one thread): S = Q.K^T (M 128, N 64, K 128) into a double-buffered
-//               TMEM tile, then O += P.V (M 128, N 128, K 64) into the piece's TMEM accumulator.
+//   warp 4      TMA producer: one 64-row x 128-B box per d-half of a page's K and V tiles
+//               (128-byte swizzle) into four rings (K d-half 0/1, V d-half 0/1) of 6 page slots;
+//               the two pages of a tile go to slots 2p and 2p+1, which are contiguous in every
+//               ring, so one descriptor spans the tile.  An odd page or the verify-token unit
+//               leaves slot 2p+1 empty.  Verify tokens come through 3-D tensor maps over
+//               k_new / v_new (16 tokens of one KV head).
+//   warp 5      MMA issuer (one thread): A operands (Q, P; bf16) in tensor memory, B operands
+//               (K, V) in shared memory, fp32 accumulators in tensor memory.
 //   warps 0-3   softmax + epilogue.  TMEM lane quadrant w is readable only by warp w, so each
-//               query row is replicated C times in the A operand (C = 4 for <= 32 rows, 2 for
-//               <= 64, 1 otherwise): copy c lives in lanes [c*128/C, (c+1)*128/C) and its warps
-//               handle keys [c*64/C, (c+1)*64/C) of every tile, which spreads the exp2 work of
-//               a row over C SM sub-partitions.  Partial row maxima are exchanged through shared
-//               memory (named barrier), P (bf16) is written to shared memory (128-byte swizzle)
-//               for the P.V MMA, and O is rescaled in TMEM only when the running maximum grows by
-//               more than 2^8.  The request's own verify tokens are one more tile at the end of
-//               the segment: TMA loads their K/V rows through 3-D tensor maps over k_new/v_new
-//               (16 tokens of one KV head) and the softmax applies the causal rule from the
-//               markers (token j sees verify tokens 0..j).  The epilogue reads O from TMEM and
-//               writes the output, or a split-KV partial that the last piece merges.
+//               query row is replicated C times (C = 4 for <= 32 rows, else 2): copy c lives in
+//               lanes [c*128/C, (c+1)*128/C) and handles keys [c*128/C, (c+1)*128/C) of every
+//               tile, spreading the exp2 work of a row over C SM sub-partitions.  Partial row
+//               maxima are exchanged through shared memory (named barrier); each copy writes P
+//               for its own keys (zeros elsewhere) into its own lanes, so every copy accumulates
+//               a partial O over its keys and the epilogue sums the copies.  O is rescaled in
+//               TMEM only when the running maximum grows by more than 2^8.  The verify-token
+//               unit applies the causal rule from the markers (token j sees verify tokens 0..j).
+// TMEM columns: S [0,256) (two 128-column tiles), Q [256,320), P [320,384), O [384,512).
 // The next piece's queries are staged as soon as the current piece's last S MMA has landed,
 // before the current epilogue, so the tensor core and TMA keep streaming across pieces.
 // Every mbarrier wait is bounded (ptx::mbar_wait); on timeout the CTA records
@@ -34,44 +42,47 @@
 namespace dspark {
 namespace tc {
 
-constexpr int kNK = 64;                              // keys per tile
-constexpr int kStages = 4;
+constexpr int kPage = 64;                            // keys per page slot
+constexpr int kTK = 128;                             // keys per tile (two page slots)
+constexpr int kSlots = 6;                            // page slots per ring (three tile pairs)
+constexpr int kPairs = kSlots / 2;
 constexpr int kThreads = 192;
 constexpr int kSoftmaxThreads = 128;
 constexpr int kD = 128;
-constexpr uint32_t kHalfTile = 64 * 128;             // 64 rows x 128 B: one d-half of a K or V tile
-constexpr uint32_t kStageBytes = 4 * kHalfTile;      // K h0 | K h1 | V h0 | V h1
-constexpr uint32_t kQBytes = 2 * 128 * 128;          // 2 d-halves x 128 A-rows x 128 B
-constexpr uint32_t kPBytes = 128 * 128;              // 128 A-rows x 64 keys x 2 B
-constexpr uint32_t kOffQ = kStages * kStageBytes;
-constexpr uint32_t kOffP = kOffQ + kQBytes;
-constexpr uint32_t kOffAux = kOffP + 2 * kPBytes;
-constexpr uint32_t kAuxBytes = 4096;
-constexpr uint32_t kSmemBytes = kOffAux + kAuxBytes + 1024;  // + 1024-B alignment slack
+constexpr int kNewRows = 16;                         // verify tokens per unit (K + 1 <= 16)
+constexpr uint32_t kSlotBytes = 64 * 128;            // 64 rows x 128 B: one d-half of a page
+constexpr uint32_t kRingBytes = kSlots * kSlotBytes; // one ring (K h0, K h1, V h0 or V h1)
+constexpr uint32_t kPageBytes = 4 * kSlotBytes;      // a full page: K and V, both d-halves
+constexpr uint32_t kNewBytes = 4 * kNewRows * 128;   // verify-token unit
+constexpr uint32_t kOffAux = 4 * kRingBytes;
+constexpr uint32_t kAuxBytes = 2048;
+constexpr uint32_t kOffScratch = kOffAux + kAuxBytes;
+constexpr uint32_t kScratchBytes = 128 * 16 * 4;     // epilogue: 128 lanes x 16 fp32
+constexpr uint32_t kSmemBytes = kOffScratch + kScratchBytes + 1024;  // + alignment slack
 
 // aux region layout (bytes)
-constexpr uint32_t kBarKvFull = 0, kBarKvEmpty = 32, kBarSFull = 64, kBarPFull = 80,
-                   kBarODone = 96, kBarQFull = 112, kBarQEmpty = 120, kBarOFree = 128;
-constexpr uint32_t kAuxTmem = 160, kAuxAbort = 164, kAuxLast = 168, kAuxPmax = 256,
+constexpr uint32_t kBarKvFull = 0, kBarKvEmpty = 64, kBarSFull = 128, kBarPFull = 144,
+                   kBarODone = 152, kBarQFull = 160, kBarQEmpty = 168, kBarOFree = 176;
+constexpr uint32_t kAuxTmem = 224, kAuxAbort = 228, kAuxLast = 232, kAuxPmax = 256,
                    kAuxLsum = 256 + 2 * 128 * 4;
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;     // S tiles: columns [0, 64) and [64, 128)
-constexpr uint32_t kColO = 256;   // O accumulators: [256, 384) and [384, 512)
+constexpr uint32_t kColS = 0;
+constexpr uint32_t kColQ = 256;
+constexpr uint32_t kColP = 320;
+constexpr uint32_t kColO = 384;
 constexpr float kRescaleLog2 = 8.f;
 
-constexpr int kNewRows = 16;                         // verify tokens per new-token tile (K + 1 <= 16)
-constexpr uint32_t kNewBytes = 4 * kNewRows * 128;   // K and V, two d-halves each
-
-constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, kNK, 0, 0);
-constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, kD, 0, 1);
+constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, kTK, 0, 0);  // Q (K-major) x K^T
+constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, kD, 0, 1);  // P (K-major) x V (MN-major)
 
 struct Meta {
-  int t0, Q, n, rows, C, ncache, ntiles;  // ntiles = cache tiles + the new-token tile
-  bool valid, last, newtile;
+  int t0, Q, n, rows, C, npages, ncache, ntiles;  // npages: cache pages of the piece
+  bool valid, last, newtile;                      // ncache: their 128-key tiles
 };
 
-// Serial validation of one piece; every role computes it identically.
+// Serial validation of one piece [ta, tb) of a segment with `tiles` units; every role computes
+// it identically.
 __device__ __forceinline__ Meta piece_meta(const AttnArgs &a, int r, int ta, int tb, int tiles,
                                            bool raise) {
   Meta m;
@@ -96,8 +107,9 @@ __device__ __forceinline__ Meta piece_meta(const AttnArgs &a, int r, int ta, int
   }
   m.valid = ok;
   m.rows = ok ? a.G * m.Q : 0;
-  m.C = m.rows <= 32 ? 4 : (m.rows <= 64 ? 2 : 1);
-  m.ncache = (ok && m.n > 0) ? (tb - ta) : 0;
+  m.C = m.rows <= 32 ? 4 : 2;
+  m.npages = ok ? max(0, min(tb, tiles - 1) - ta) : 0;
+  m.ncache = (m.npages + 1) / 2;
   m.last = (tb == tiles);
   m.newtile = ok && m.last;
   m.ntiles = m.ncache + (m.newtile ? 1 : 0);
@@ -142,18 +154,19 @@ struct SoftmaxState {
   float l_part;  // partial row sum over this copy's keys
 };
 
-// One tile for the thread's A-row t: S slice from TMEM, masking, row maximum across copies
-// (named barrier 1), conditional O rescale, P (bf16) into shared memory.  NKC = keys per copy.
+// One tile for the thread's lane: S slice from TMEM, masking (valid keys, causal bound), row
+// maximum across copies (named barrier 1), conditional rescale of this lane's O, P (bf16) for
+// this copy's keys into this lane's P columns.  NKC = keys per copy.  `gt` = global tile index.
 template <int NKC>
 __device__ __forceinline__ void softmax_tile(const AttnArgs &a, SoftmaxState &st, uint32_t tmem,
-                                             uint32_t lane_base, uint32_t base, uint32_t aux,
-                                             float *pmax_buf, volatile int *abort_flag,
-                                             uint32_t g_, int vk, int jrow, int t, int copy,
-                                             int rho, int rpc, bool active, uint32_t ob) {
-  constexpr int C = kNK / NKC;
-  const uint32_t b = g_ & 1;
+                                             uint32_t lane_base, uint32_t aux, float *pmax_buf,
+                                             volatile int *abort_flag, uint32_t gt, int vk,
+                                             int jrow, int t, int copy, int rho, int rpc,
+                                             bool active) {
+  constexpr int C = kTK / NKC;
+  const uint32_t b = gt & 1;
   float s[NKC];
-  const uint32_t s_taddr = tmem + lane_base + kColS + b * kNK + copy * NKC;
+  const uint32_t s_taddr = tmem + lane_base + kColS + b * kTK + copy * NKC;
 #pragma unroll
   for (int c16 = 0; c16 < NKC / 16; ++c16) {
     float v[16];
@@ -166,7 +179,7 @@ __device__ __forceinline__ void softmax_tile(const AttnArgs &a, SoftmaxState &st
 #pragma unroll
   for (int i = 0; i < NKC; ++i) {
     const int key = copy * NKC + i;
-    const float x = (key < vk && key <= jrow) ? s[i] * a.scale_log2 : -INFINITY;
+    const float x = (active && key < vk && key <= jrow) ? s[i] * a.scale_log2 : -INFINITY;
     s[i] = x;
     mx = fmaxf(mx, x);
   }
@@ -186,46 +199,39 @@ __device__ __forceinline__ void softmax_tile(const AttnArgs &a, SoftmaxState &st
     st.l_part *= alpha;
     resc = true;
   }
-  if (copy == 0 && __any_sync(0xffffffffu, resc)) {
-    // O holds the earlier tiles relative to the old maximum: rescale it in TMEM once the
-    // previous P.V has landed
-    const uint32_t gp = g_ - 1;
-    ptx::mbar_wait(aux + kBarODone + 8u * (gp & 1), (gp >> 1) & 1, abort_flag);
-    ptx::tc_fence_after();
-    const uint32_t o_taddr = tmem + lane_base + kColO + ob * 128;
-#pragma unroll 1
-    for (int c16 = 0; c16 < 8; ++c16) {
-      float v[16];
-      ptx::tmem_ld16(o_taddr + c16 * 16, v);
-      ptx::tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] *= alpha;
-      ptx::tmem_st16(o_taddr + c16 * 16, v);
-    }
-    ptx::tmem_wait_st();
-  }
-  // P buffer b was last read by the P.V of tile g_ - 2
-  if (g_ >= 2) ptx::mbar_wait(aux + kBarODone + 8u * b, ((g_ - 2) >> 1) & 1, abort_flag);
-  const uint32_t p_row = base + kOffP + b * kPBytes + (uint32_t)rho * 128;
+  // compute P before waiting for the tensor core
   float lsum = 0.f;
+  uint32_t w[NKC / 2];
 #pragma unroll
-  for (int c8 = 0; c8 < NKC / 8; ++c8) {
-    uint32_t w4[4];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const float p0 = ex2(s[c8 * 8 + 2 * h] - st.m_run);
-      const float p1 = ex2(s[c8 * 8 + 2 * h + 1] - st.m_run);
-      const __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
-      const float2 back = __bfloat1622float2(hb);
-      lsum += back.x + back.y;
-      w4[h] = *reinterpret_cast<const uint32_t *>(&hb);
-    }
-    if (active) {
-      const uint32_t kc = (uint32_t)(copy * (NKC / 8) + c8);
-      st_shared_v4(p_row + ((kc ^ ((uint32_t)rho & 7)) << 4), w4[0], w4[1], w4[2], w4[3]);
-    }
+  for (int h = 0; h < NKC / 2; ++h) {
+    const float p0 = active ? ex2(s[2 * h] - st.m_run) : 0.f;
+    const float p1 = active ? ex2(s[2 * h + 1] - st.m_run) : 0.f;
+    const __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+    const float2 back = __bfloat1622float2(hb);
+    lsum += back.x + back.y;
+    w[h] = *reinterpret_cast<const uint32_t *>(&hb);
   }
   st.l_part += lsum;
+  // the single P tile and this lane's O were last used by the P.V of tile gt - 1
+  if (gt >= 1) {
+    ptx::mbar_wait(aux + kBarODone, (gt - 1) & 1, abort_flag);
+    ptx::tc_fence_after();
+  }
+  if (__any_sync(0xffffffffu, resc)) {
+    // this lane's O holds the earlier tiles relative to the old maximum: rescale it in TMEM
+    const uint32_t o_taddr = tmem + lane_base + kColO;
+#pragma unroll 1
+    for (int c32 = 0; c32 < 4; ++c32) {
+      float v[32];
+      ptx::tmem_ld32(o_taddr + c32 * 32, v);
+      ptx::tmem_wait_ld();
+      uint32_t ow[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ow[i] = __float_as_uint(v[i] * alpha);
+      ptx::tmem_st<32>(o_taddr + c32 * 32, ow);
+    }
+  }
+  ptx::tmem_st<NKC / 2>(tmem + lane_base + kColP + copy * (NKC / 2), w);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -241,24 +247,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
   volatile int *abort_flag = reinterpret_cast<volatile int *>(gaux + kAuxAbort);
   float *pmax_buf = reinterpret_cast<float *>(gaux + kAuxPmax);
   float *lsum_buf = reinterpret_cast<float *>(gaux + kAuxLsum);
+  float *scratch = reinterpret_cast<float *>(gbase + kOffScratch);
   volatile int *s_last = reinterpret_cast<volatile int *>(gaux + kAuxLast);
+  // ring r (0 = K d-half 0, 1 = K d-half 1, 2 = V d-half 0, 3 = V d-half 1), page slot s
+  auto ring = [&](int rg, uint32_t s) { return base + (uint32_t)rg * kRingBytes + s * kSlotBytes; };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   auto bar = [&](uint32_t off, int i) { return aux + off + 8u * (uint32_t)i; };
 
   if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kSlots; ++i) {
       ptx::mbar_init(bar(kBarKvFull, i), 1);
       ptx::mbar_init(bar(kBarKvEmpty, i), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(bar(kBarSFull, i), 1);
-      ptx::mbar_init(bar(kBarPFull, i), kSoftmaxThreads);
-      ptx::mbar_init(bar(kBarODone, i), 1);
-      ptx::mbar_init(bar(kBarOFree, i), kSoftmaxThreads);
-    }
+    for (int i = 0; i < 2; ++i) ptx::mbar_init(bar(kBarSFull, i), 1);
+    ptx::mbar_init(bar(kBarPFull, 0), kSoftmaxThreads);
+    ptx::mbar_init(bar(kBarODone, 0), 1);
     ptx::mbar_init(bar(kBarQFull, 0), kSoftmaxThreads);
     ptx::mbar_init(bar(kBarQEmpty, 0), 1);
+    ptx::mbar_init(bar(kBarOFree, 0), kSoftmaxThreads);
     *abort_flag = 0;
     *s_last = 0;
     ptx::fence_mbar_init();
@@ -284,95 +291,106 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
   if (warp == 4) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t gt = 0, issued = 0;
+      uint32_t gs = 0;  // global page-slot counter (slot = gs % kSlots), always even per tile
+      int last_use[kSlots];  // latest slot use that was armed (TMA or empty arrive), -1 if none
+#pragma unroll
+      for (int k = 0; k < kSlots; ++k) last_use[k] = -1;
+      auto wait_slot = [&](uint32_t sl) {
+        ptx::mbar_wait(bar(kBarKvEmpty, sl % kSlots), ((sl / kSlots) & 1) ^ 1, abort_flag);
+      };
       while (it.next(a, r, g, ta, tb, tiles, s0)) {
         const Meta m = piece_meta(a, r, ta, tb, tiles, false);
-        for (int j = 0; j < m.ntiles; ++j, ++gt) {
-          const uint32_t st = gt % kStages;
-          ptx::mbar_wait(bar(kBarKvEmpty, st), ((gt / kStages) & 1) ^ 1, abort_flag);
-          if (*abort_flag) continue;
-          const uint32_t sb = base + st * kStageBytes;
-          const uint32_t fb = bar(kBarKvFull, st);
-          if (j < m.ncache) {
-            const int key0 = (ta + j) * kNK;
-            const int page = __ldg(a.block_table + (size_t)r * a.max_pages + key0 / a.page_size);
-            int rowK = oob_row, rowV = oob_row;
-            if (page >= 0 && page < a.num_pages) {
-              rowK = ((page * 2) * a.Hkv + g) * a.page_size + key0 % a.page_size;
-              rowV = rowK + a.Hkv * a.page_size;
+        for (int j = 0; j < m.ntiles; ++j, gs += 2) {
+          for (int h = 0; h < 2; ++h) {   // the tile's two page slots
+            const uint32_t sl = gs + h, slot = sl % kSlots;
+            wait_slot(sl);
+            if (*abort_flag) continue;
+            const uint32_t fb = bar(kBarKvFull, slot);
+            const int pg = 2 * j + h;     // page of the piece in this slot
+            if (j < m.ncache && pg < m.npages) {
+              const int key0 = (ta + pg) * kPage;
+              const int page = __ldg(a.block_table + (size_t)r * a.max_pages + key0 / a.page_size);
+              int rowK = oob_row, rowV = oob_row;
+              if (page >= 0 && page < a.num_pages) {
+                rowK = ((page * 2) * a.Hkv + g) * a.page_size + key0 % a.page_size;
+                rowV = rowK + a.Hkv * a.page_size;
+              } else {
+                raise_error(DSPARK_DERR_PAGE);
+              }
+              ptx::mbar_arrive_expect_tx(fb, kPageBytes);
+              ptx::tma_load_2d(ring(0, slot), &tmap_kv, fb, 0, rowK);
+              ptx::tma_load_2d(ring(1, slot), &tmap_kv, fb, 64, rowK);
+              ptx::tma_load_2d(ring(2, slot), &tmap_kv, fb, 0, rowV);
+              ptx::tma_load_2d(ring(3, slot), &tmap_kv, fb, 64, rowV);
+            } else if (j == m.ncache && h == 0) {  // the verify tokens: 16 rows of KV head g
+              ptx::mbar_arrive_expect_tx(fb, kNewBytes);
+              ptx::tma_load_3d(ring(0, slot), &tmap_kn, fb, 0, g, m.t0);
+              ptx::tma_load_3d(ring(1, slot), &tmap_kn, fb, 64, g, m.t0);
+              ptx::tma_load_3d(ring(2, slot), &tmap_vn, fb, 0, g, m.t0);
+              ptx::tma_load_3d(ring(3, slot), &tmap_vn, fb, 64, g, m.t0);
             } else {
-              raise_error(DSPARK_DERR_PAGE);
+              ptx::mbar_arrive(fb);  // empty slot: completes its phase without data
             }
-            ptx::mbar_arrive_expect_tx(fb, kStageBytes);
-            ptx::tma_load_2d(sb, &tmap_kv, fb, 0, rowK);
-            ptx::tma_load_2d(sb + kHalfTile, &tmap_kv, fb, 64, rowK);
-            ptx::tma_load_2d(sb + 2 * kHalfTile, &tmap_kv, fb, 0, rowV);
-            ptx::tma_load_2d(sb + 3 * kHalfTile, &tmap_kv, fb, 64, rowV);
-          } else {  // the request's own verify tokens: 16 token rows of KV head g
-            ptx::mbar_arrive_expect_tx(fb, kNewBytes);
-            ptx::tma_load_3d(sb, &tmap_kn, fb, 0, g, m.t0);
-            ptx::tma_load_3d(sb + kHalfTile, &tmap_kn, fb, 64, g, m.t0);
-            ptx::tma_load_3d(sb + 2 * kHalfTile, &tmap_vn, fb, 0, g, m.t0);
-            ptx::tma_load_3d(sb + 3 * kHalfTile, &tmap_vn, fb, 64, g, m.t0);
+            last_use[slot] = (int)sl;
           }
-          issued = gt + 1;
         }
       }
-      // never leave the CTA with a bulk copy in flight: wait for the last use of every stage
+      // never leave the CTA with a bulk copy in flight: wait for the latest armed use of every
+      // slot (its phase is the newest one the slot's barrier can complete)
       volatile int no_abort = 0;
-      for (uint32_t k = 0; k < kStages && k < issued; ++k) {
-        const uint32_t g_ = issued - 1 - k;
-        ptx::mbar_wait(bar(kBarKvFull, g_ % kStages), (g_ / kStages) & 1, &no_abort);
-      }
+      for (int k = 0; k < kSlots; ++k)
+        if (last_use[k] >= 0)
+          ptx::mbar_wait(bar(kBarKvFull, k), ((uint32_t)last_use[k] / kSlots) & 1, &no_abort);
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t gt = 0, pq = 0;
+      uint32_t gt = 0, pq = 0;  // global tile counter, pieces with tiles
       while (it.next(a, r, g, ta, tb, tiles, s0)) {
         const Meta m = piece_meta(a, r, ta, tb, tiles, false);
         if (m.ntiles == 0) continue;
-        const uint32_t ob = pq & 1;
         ptx::mbar_wait(bar(kBarQFull, 0), pq & 1, abort_flag);
-        ptx::mbar_wait(bar(kBarOFree, ob), ((pq >> 1) & 1) ^ 1, abort_flag);
         ptx::tc_fence_after();
-        const uint32_t q_addr = base + kOffQ;
-        auto issue_pv = [&](uint32_t g_, int jj) {
-          ptx::mbar_wait(bar(kBarPFull, g_ & 1), (g_ >> 1) & 1, abort_flag);
+        auto issue_pv = [&](uint32_t gt_, int jj) {
+          if (jj == 0) {  // O of the previous piece has been read by its epilogue
+            ptx::mbar_wait(bar(kBarOFree, 0), (pq & 1) ^ 1, abort_flag);
+          }
+          ptx::mbar_wait(bar(kBarPFull, 0), gt_ & 1, abort_flag);
           ptx::tc_fence_after();
           if (*abort_flag) return;
-          const uint32_t p_addr = base + kOffP + (g_ & 1) * kPBytes;
-          const uint32_t v_addr = base + (g_ % kStages) * kStageBytes + 2 * kHalfTile;
-          const uint32_t d_tmem = tmem + kColO + ob * 128;
-          const int ksteps = (jj < m.ncache) ? kNK / 16 : kNewRows / 16;
+          const uint32_t pair = gt_ % kPairs;
+          const int ksteps = (jj < m.ncache) ? (min(kTK, m.npages * kPage - jj * kTK) / 16)
+                                             : kNewRows / 16;
           for (int k = 0; k < ksteps; ++k) {
-            const uint64_t ad = ptx::smem_desc_sw128(p_addr + k * 32, 16, 1024);
-            const uint64_t bd = ptx::smem_desc_sw128(v_addr + k * 2048, kHalfTile, 1024);
-            ptx::mma_bf16_ss(d_tmem, ad, bd, kIdescPV, (jj > 0 || k > 0) ? 1u : 0u);
+            const uint64_t bd =
+                ptx::smem_desc_sw128(ring(2, 2 * pair) + k * 2048, kRingBytes, 1024);
+            ptx::mma_bf16_ts(tmem + kColO, tmem + kColP + k * 8, bd, kIdescPV,
+                             (jj > 0 || k > 0) ? 1u : 0u);
           }
-          ptx::mma_commit(bar(kBarODone, g_ & 1));
-          ptx::mma_commit(bar(kBarKvEmpty, g_ % kStages));
+          ptx::mma_commit(bar(kBarODone, 0));
+          ptx::mma_commit(bar(kBarKvEmpty, 2 * pair));
+          ptx::mma_commit(bar(kBarKvEmpty, 2 * pair + 1));
         };
         for (int j = 0; j < m.ntiles; ++j) {
-          const uint32_t g_ = gt + j;
-          const uint32_t st = g_ % kStages;
-          ptx::mbar_wait(bar(kBarKvFull, st), (g_ / kStages) & 1, abort_flag);
+          const uint32_t gt_ = gt + j;
+          const uint32_t pair = gt_ % kPairs;
+          const uint32_t ph = (gt_ / kPairs) & 1;
+          ptx::mbar_wait(bar(kBarKvFull, 2 * pair), ph, abort_flag);
+          ptx::mbar_wait(bar(kBarKvFull, 2 * pair + 1), ph, abort_flag);
           ptx::tc_fence_after();
           if (!*abort_flag) {
-            const uint32_t k_addr = base + st * kStageBytes;
-            const uint32_t d_tmem = tmem + kColS + (g_ & 1) * kNK;
+            const uint32_t d_tmem = tmem + kColS + (gt_ & 1) * kTK;
 #pragma unroll
             for (int k = 0; k < kD / 16; ++k) {
               const uint32_t h = k >> 2, kk = k & 3;
-              const uint64_t ad = ptx::smem_desc_sw128(q_addr + h * 16384 + kk * 32, 16, 1024);
-              const uint64_t bd = ptx::smem_desc_sw128(k_addr + h * kHalfTile + kk * 32, 16, 1024);
-              ptx::mma_bf16_ss(d_tmem, ad, bd, kIdescS, k > 0 ? 1u : 0u);
+              const uint64_t bd = ptx::smem_desc_sw128(ring(h, 2 * pair) + kk * 32, 16, 1024);
+              ptx::mma_bf16_ts(d_tmem, tmem + kColQ + k * 8, bd, kIdescS, k > 0 ? 1u : 0u);
             }
-            ptx::mma_commit(bar(kBarSFull, g_ & 1));
+            ptx::mma_commit(bar(kBarSFull, gt_ & 1));
             // the piece's last S read of Q: the next piece may stage its queries
             if (j == m.ntiles - 1) ptx::mma_commit(bar(kBarQEmpty, 0));
           }
-          if (j > 0) issue_pv(g_ - 1, j - 1);
+          if (j > 0) issue_pv(gt_ - 1, j - 1);
         }
         issue_pv(gt + m.ntiles - 1, m.ntiles - 1);
         gt += m.ntiles;
@@ -380,36 +398,44 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       }
       if (gt > 0 && !*abort_flag) {  // every MMA of this CTA has completed before TMEM is released
         volatile int no_abort = 0;
-        ptx::mbar_wait(bar(kBarODone, (gt - 1) & 1), ((gt - 1) >> 1) & 1, &no_abort);
+        ptx::mbar_wait(bar(kBarODone, 0), (gt - 1) & 1, &no_abort);
       }
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    const int t = tid;  // A-row of this thread (0..127)
+    const int t = tid;  // TMEM lane of this thread (0..127)
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(a.q);
     __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.out);
     const int G = a.G;
-    uint32_t gt = 0, pq = 0, qidx = 0;
+    uint32_t gt = 0, qidx = 0;
 
-    // queries of a piece, replicated per copy, into the Q buffer once the previous piece's
-    // last S MMA no longer reads it
+    // A piece's queries, replicated per copy, into this lane's Q columns once the previous
+    // piece's last S MMA no longer reads them (inactive lanes get zeros).
     auto stage_q = [&](const Meta &mq, int gq) {
       const int rpcq = 128 / mq.C, rq = t % rpcq;
       ptx::mbar_wait(bar(kBarQEmpty, 0), (qidx & 1) ^ 1, abort_flag);
-      if (rq < mq.rows) {
-        const int j = rq / G, i = rq % G;
-        const uint4 *src = reinterpret_cast<const uint4 *>(
-            qg + ((size_t)(mq.t0 + j) * a.Hq + gq * G + i) * kD);
+      ptx::tc_fence_after();
+      uint32_t w[32];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const uint4 v = __ldg(src + c);
-          const uint32_t addr = base + kOffQ + (c >> 3) * 16384 + t * 128 +
-                                ((((uint32_t)c & 7) ^ ((uint32_t)t & 7)) << 4);
-          st_shared_v4(addr, v.x, v.y, v.z, v.w);
+      for (int h = 0; h < 2; ++h) {
+        if (rq < mq.rows) {
+          const int j = rq / G, i = rq % G;
+          const uint4 *src = reinterpret_cast<const uint4 *>(
+              qg + ((size_t)(mq.t0 + j) * a.Hq + gq * G + i) * kD + h * 64);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = __ldg(src + c);
+            w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) w[c] = 0u;
         }
+        ptx::tmem_st<32>(tmem + lane_base + kColQ + h * 32, w);
       }
-      ptx::fence_proxy_async_smem();
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
       ptx::mbar_arrive(bar(kBarQFull, 0));
       ++qidx;
     };
@@ -421,44 +447,51 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       if (m.ntiles > 0) stage_q(m, g);
     }
     while (have) {
-      const int rpc = 128 / m.C;         // A-rows per copy
+      const int rpc = 128 / m.C;         // lanes per copy
       const int copy = t / rpc, rho = t % rpc;
       const bool active = m.valid && rho < m.rows;
       SoftmaxState sm;
       sm.m_run = -INFINITY;
       sm.l_part = 0.f;
-      const uint32_t ob = pq & 1;
       for (int j = 0; j < m.ntiles; ++j) {
-        const uint32_t g_ = gt + j;
-        const uint32_t b = g_ & 1;
+        const uint32_t gt_ = gt + j;
         const bool cache_tile = j < m.ncache;
-        const int vk = cache_tile ? min(kNK, m.n - (ta + j) * kNK) : m.Q;  // valid keys
-        const int jrow = cache_tile ? 0x7fffffff : rho / G;                // causal bound
-        ptx::mbar_wait(bar(kBarSFull, b), (g_ >> 1) & 1, abort_flag);
+        // valid keys: the tile's pages that belong to this piece, cut at the cache length
+        const int vk = cache_tile ? min(min(2, m.npages - 2 * j) * kPage, m.n - (ta + 2 * j) * kPage)
+                                  : m.Q;
+        const int jrow = cache_tile ? 0x7fffffff : rho / G;                      // causal bound
+        ptx::mbar_wait(bar(kBarSFull, gt_ & 1), (gt_ >> 1) & 1, abort_flag);
         ptx::tc_fence_after();
+        if (j == 0) {
+          // this lane's P columns outside its copy's keys must read as zero (the previous
+          // piece's P.V MMAs have completed: its epilogue waited for them)
+          uint32_t z[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) z[c] = 0u;
+          ptx::tmem_st<32>(tmem + lane_base + kColP, z);
+          ptx::tmem_st<32>(tmem + lane_base + kColP + 32, z);
+        }
         if (m.C == 4)
-          softmax_tile<16>(a, sm, tmem, lane_base, base, aux, pmax_buf, abort_flag, g_, vk, jrow,
-                           t, copy, rho, rpc, active, ob);
-        else if (m.C == 2)
-          softmax_tile<32>(a, sm, tmem, lane_base, base, aux, pmax_buf, abort_flag, g_, vk, jrow,
-                           t, copy, rho, rpc, active, ob);
+          softmax_tile<32>(a, sm, tmem, lane_base, aux, pmax_buf, abort_flag, gt_, vk, jrow, t,
+                           copy, rho, rpc, active);
         else
-          softmax_tile<64>(a, sm, tmem, lane_base, base, aux, pmax_buf, abort_flag, g_, vk, jrow,
-                           t, copy, rho, rpc, active, ob);
-        const int vrows = cache_tile ? kNK : kNewRows;  // V rows the P.V MMA reads
+          softmax_tile<64>(a, sm, tmem, lane_base, aux, pmax_buf, abort_flag, gt_, vk, jrow, t,
+                           copy, rho, rpc, active);
+        // V rows the P.V MMA reads past the valid keys may hold anything: zero them so that
+        // P = 0 times V stays 0 (the MMA reads whole 16-key steps of valid pages)
+        const int vrows = cache_tile ? min(kTK, (vk + kPage - 1) / kPage * kPage) : kNewRows;
         if (vk < vrows) {
-          // keys past the valid ones: their V rows may hold anything; zero them so that
-          // P = 0 times V stays 0
-          ptx::mbar_wait(bar(kBarKvFull, g_ % kStages), (g_ / kStages) & 1, abort_flag);
-          const uint32_t v_addr = base + (g_ % kStages) * kStageBytes + 2 * kHalfTile;
+          const uint32_t pair = gt_ % kPairs;
+          ptx::mbar_wait(bar(kBarKvFull, 2 * pair + vk / kPage), (gt_ / kPairs) & 1, abort_flag);
           for (int idx = t; idx < (vrows - vk) * 16; idx += kSoftmaxThreads) {
             const uint32_t row = vk + idx / 16, half = (idx % 16) / 8, c = idx % 8;
-            st_shared_v4(v_addr + half * kHalfTile + row * 128 + c * 16, 0u, 0u, 0u, 0u);
+            st_shared_v4(ring(2 + half, 2 * pair) + row * 128 + c * 16, 0u, 0u, 0u, 0u);
           }
+          ptx::fence_proxy_async_smem();
         }
-        ptx::fence_proxy_async_smem();
+        ptx::tmem_wait_st();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(bar(kBarPFull, b));
+        ptx::mbar_arrive(bar(kBarPFull, 0));
       }
 
       // stage the next piece's queries now, so the MMAs of the next piece overlap this epilogue
@@ -472,29 +505,44 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
 
       // ---------------------------------------------------------------- epilogue
       lsum_buf[t] = sm.l_part;
-      ptx::named_bar_sync(2, kSoftmaxThreads);
       if (m.ntiles > 0) {
-        const uint32_t gl = gt + m.ntiles - 1;
-        ptx::mbar_wait(bar(kBarODone, gl & 1), (gl >> 1) & 1, abort_flag);
+        ptx::mbar_wait(bar(kBarODone, 0), (gt + m.ntiles - 1) & 1, abort_flag);
         ptx::tc_fence_after();
       }
+      ptx::named_bar_sync(2, kSoftmaxThreads);
       const bool whole = (ta == 0 && tb == tiles);
       const int W = it.W;
       float *part = a.ws.partials +
                     (size_t)partial_slot(blockIdx.x, s0, W) * a.rows_max * (kD + 2);
-      if (copy == 0 && m.ntiles > 0) {  // warp-uniform: copy-0 warps own the O rows
+      if (m.ntiles > 0) {
         float l = 0.f;
         for (int cc = 0; cc < m.C; ++cc) l += lsum_buf[rho + cc * rpc];
-        const int j = active ? rho / G : 0, i = active ? rho % G : 0;
-        const size_t orow = ((size_t)(m.t0 + j) * a.Hq + g * G + i) * kD;
-        const uint32_t o_taddr = tmem + lane_base + kColO + ob * 128;
         const float inv = 1.f / l;
+        const int j = rho / G, i = rho % G;
+        const size_t orow = ((size_t)(m.t0 + j) * a.Hq + g * G + i) * kD;
+        const uint32_t o_taddr = tmem + lane_base + kColO;
 #pragma unroll 1
         for (int c16 = 0; c16 < 8; ++c16) {
           float o[16];
-          ptx::tmem_ld16(o_taddr + c16 * 16, o);
+          ptx::tmem_ld16(o_taddr + c16 * 16, o);  // this copy's partial O
           ptx::tmem_wait_ld();
-          if (active) {
+          // sum the copies' partial O rows through shared memory
+          float4 *sv = reinterpret_cast<float4 *>(scratch + t * 16);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sv[e] = make_float4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+          ptx::named_bar_sync(2, kSoftmaxThreads);
+          if (copy == 0) {
+            for (int cc = 1; cc < m.C; ++cc) {
+              const float4 *sv2 = reinterpret_cast<const float4 *>(scratch + (rho + cc * rpc) * 16);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float4 x = sv2[e];
+                o[4 * e] += x.x; o[4 * e + 1] += x.y; o[4 * e + 2] += x.z; o[4 * e + 3] += x.w;
+              }
+            }
+          }
+          ptx::named_bar_sync(2, kSoftmaxThreads);
+          if (active && copy == 0) {
             if (whole) {
               uint32_t w8[8];
 #pragma unroll
@@ -510,16 +558,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
             }
           }
         }
-        if (active && !whole) {
+        if (active && copy == 0 && !whole) {
           part[(size_t)rho * (kD + 2) + kD] = sm.m_run;
           part[(size_t)rho * (kD + 2) + kD + 1] = l;
         }
-      }
-      if (m.ntiles > 0) {
         ptx::tc_fence_before();
-        ptx::mbar_arrive(bar(kBarOFree, ob));
+        ptx::mbar_arrive(bar(kBarOFree, 0));
         gt += m.ntiles;
-        ++pq;
       }
 
       if (!whole) {  // split segment: publish the partial, the last piece merges

@@ -201,7 +201,7 @@ int dspark_verify_attn(const void *q, const void *k_new, const void *v_new, cons
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const uint64_t kv_rows = (uint64_t)num_pages * 2 * Hkv * page_size;
   if (dtype == DSPARK_BF16 && D == 128 && page_size % 64 == 0 && kv_rows < (1ull << 31) &&
-      K + 1 <= tc::kNewRows) {
+      K + 1 <= tc::kNewRows && rows_max <= 64) {
     CUtensorMap map, map_kn, map_vn;
     if (!encode_kv_map(&map, kv_pages, kv_rows) || !encode_new_map(&map_kn, k_new, T_cap, Hkv) ||
         !encode_new_map(&map_vn, v_new, T_cap, Hkv))
