@@ -128,18 +128,25 @@ int dspark_schedule(const float *conf_ring, int ring_depth, int round_idx, int R
 size_t dspark_verify_attn_workspace_bytes(int R, int Hq, int Hkv, int D, int K);
 
 /*
- * dspark_verify_attn_plan — partition one step's attention work across the GPU.
+ * dspark_verify_attn_plan — partition one step's attention work across the GPU and check the
+ * flattened batch once.
  *
  * Work is the sequence of (request r, KV head g, unit) in request-major order, each request
- * contributing Hkv * (ceil(kv_len[r] / 64) + 1) units (its 64-key cache tiles, then its own
- * verify tokens); the plan splits it into
- * equal contiguous ranges, one per persistent CTA.  Call once per step after the schedule
- * (the partition depends only on kv_len and the request count), before any
- * dspark_verify_attn of that step; it also zeroes the workspace's arrival counters.
- * kv_len int32 [R] (device); ws/ws_bytes as returned by the query above.
+ * contributing Hkv * (ceil(kv_len[r] / 64) + 8) units (its 64-key cache tiles, then eight
+ * units standing for its own verify tokens and the segment's epilogue, which cost about as much
+ * as eight cache tiles); the plan splits it into equal contiguous ranges, one per persistent CTA.
+ * It also records, per request, the flattened offset, the token count and whether the
+ * flattening is well formed (1 <= Q_r <= K + 1 tokens inside [0, T_cap), token j carrying the
+ * marker (r, kv_len[r] + j)); a malformed request sets DSPARK_DERR_OFFSETS / _MARKER here and
+ * every dspark_verify_attn that uses this plan skips it.  Call once per step after the
+ * schedule and before any dspark_verify_attn of that step, and again whenever kv_len,
+ * q_offsets or markers change; it also zeroes the workspace's arrival counters.
+ * kv_len int32 [R], q_offsets int32 [R + 1], markers int32 [T_cap][2] (device); ws/ws_bytes as
+ * returned by the query above.
  */
-int dspark_verify_attn_plan(const int32_t *kv_len, int R, int Hq, int Hkv, int D, int K,
-                            void *ws, size_t ws_bytes, dspark_stream_t stream);
+int dspark_verify_attn_plan(const int32_t *kv_len, const int32_t *q_offsets,
+                            const int32_t *markers, int R, int T_cap, int Hq, int Hkv, int D,
+                            int K, void *ws, size_t ws_bytes, dspark_stream_t stream);
 
 /*
  * dspark_verify_attn — flattened ragged GQA attention of every verify token.

@@ -3,8 +3,8 @@
 // The flattened verify batch ("刚融完500亿…专治AI“嘴慢”", engineering table row "内核利用率暴跌":
 // every verify token is an independent element, no per-request padding) is turned into a
 // sequence of work units: for each request r (in order) and each KV head g, the request's cache
-// is cut into tiles of kTileKeys positions, followed by one unit for the request's own verify
-// tokens (so a request with an empty cache still has one unit).  A segment = all units of one
+// is cut into tiles of kTileKeys positions, followed by kSegTail units standing for the request's
+// own verify tokens (so a request with an empty cache still has work units).  A segment = all units of one
 // (r, g); all G*Q_r query rows of the segment are processed together, so every KV byte is read
 // once.
 //
@@ -29,11 +29,15 @@ struct AttnPlanHeader {
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Floats per row of a split-KV partial: acc[D], then m and l, padded so rows stay 16-byte aligned.
+__host__ __device__ constexpr int part_stride(int D) { return D + 4; }
+
 struct AttnWs {
   AttnPlanHeader *hdr;
   int *tile_prefix;  // [R + 1]: first unit of request r (units of all its Hkv segments)
   int *counters;     // [R * Hkv] arrival counters of split segments (kept at zero between calls)
-  float *partials;   // [2 * max_ctas][rows_max][D + 2]: acc[D], m, l per row
+  int4 *req;         // [R]: per request {t0, Q, kv_len, schedule valid} written by the plan
+  float *partials;   // [2 * max_ctas][rows_max][part_stride(D)]: acc[D], m, l per row
 };
 
 __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, int D,
@@ -42,25 +46,43 @@ __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, i
   const size_t o_hdr = off;                off += align256(sizeof(AttnPlanHeader));
   const size_t o_pre = off;                off += align256((size_t)(R + 1) * sizeof(int));
   const size_t o_cnt = off;                off += align256((size_t)R * Hkv * sizeof(int));
+  const size_t o_req = off;                off += align256((size_t)R * sizeof(int4));
   const size_t o_par = off;
-  off += align256((size_t)2 * max_ctas * rows_max * (D + 2) * sizeof(float));
+  off += align256((size_t)2 * max_ctas * rows_max * part_stride(D) * sizeof(float));
   if (ws) {
     char *b = static_cast<char *>(base);
     ws->hdr = reinterpret_cast<AttnPlanHeader *>(b + o_hdr);
     ws->tile_prefix = reinterpret_cast<int *>(b + o_pre);
     ws->counters = reinterpret_cast<int *>(b + o_cnt);
+    ws->req = reinterpret_cast<int4 *>(b + o_req);
     ws->partials = reinterpret_cast<float *>(b + o_par);
   }
   return off;
 }
 
-// Units of one (request, KV head) segment: cache tiles plus the verify-token unit.
-__host__ __device__ inline int segment_units(int n) { return (n + kTileKeys - 1) / kTileKeys + 1; }
+// Units of one (request, KV head) segment: one per 64-key cache tile, then kSegTail units for
+// the verify tokens.  The verify tokens are one tile of work plus the segment's epilogue and the
+// pipeline refill of the next segment, which together cost about as much time as eight cache
+// tiles (measured: a weight of 1, 3, 5, 8 gave 183, 167, 150, 140 us on 64 requests of 512..4096
+// cached keys), so the tail is weighted that way for the equal split across CTAs.  A CTA range that covers only tail units of a segment (not its last
+// unit) is an empty piece: it contributes a partial with no keys.
+constexpr int kSegTail = 8;
+__host__ __device__ inline int segment_units(int n) {
+  return (n + kTileKeys - 1) / kTileKeys + kSegTail;
+}
+// Cache tiles of a segment with `units` units.
+__host__ __device__ inline int segment_cache_tiles(int units) { return units - kSegTail; }
 
-// Plan: tile_prefix (exclusive scan of Hkv * segment_units(kv_len)) and counters = 0.
+// Plan: tile_prefix (exclusive scan of Hkv * segment_units(kv_len)), counters = 0, and one
+// record per request: its flattened offset t0, token count Q, cache length, and whether the
+// flattening is well formed (1 <= Q <= K + 1 inside [0, T_cap), and token j of the request
+// carries the marker (r, kv_len + j) — the layout the scheduler's flattening step produces).
+// A malformed request raises its error bit here, once per step, and is skipped by the
+// attention calls that use this plan.
 __global__ void __launch_bounds__(1024)
-attn_plan_kernel(const int32_t *__restrict__ kv_len, int R, int Hkv, int rows_max, int D,
-                 AttnWs ws) {
+attn_plan_kernel(const int32_t *__restrict__ kv_len, const int32_t *__restrict__ q_offsets,
+                 const int32_t *__restrict__ markers, int R, int T_cap, int K, int Hkv,
+                 int rows_max, int D, AttnWs ws) {
   __shared__ int warp_tot[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = (R + blockDim.x - 1) / blockDim.x;
@@ -100,6 +122,20 @@ attn_plan_kernel(const int32_t *__restrict__ kv_len, int R, int Hkv, int rows_ma
     }
   }
   for (int i = tid; i < R * Hkv; i += blockDim.x) ws.counters[i] = 0;
+  for (int r = tid; r < R; r += blockDim.x) {
+    const int t0 = q_offsets[r], Q = q_offsets[r + 1] - t0, n = kv_len[r];
+    bool ok = Q >= 1 && Q <= K + 1 && t0 >= 0 && t0 <= T_cap - Q;
+    if (!ok) raise_error(DSPARK_DERR_OFFSETS);
+    ok = ok && n >= 0;
+    if (ok) {
+      bool good = true;
+      for (int j = 0; j < Q; ++j)
+        good &= (markers[2 * (t0 + j)] == r) & (markers[2 * (t0 + j) + 1] == n + j);
+      if (!good) raise_error(DSPARK_DERR_MARKER);
+      ok = good;
+    }
+    ws.req[r] = make_int4(t0, Q, n, ok ? 1 : 0);
+  }
   if (tid == 0) {
     ws.hdr->R = R;
     ws.hdr->Hkv = Hkv;

@@ -158,7 +158,7 @@ attn_generic_kernel(AttnArgs a) {
     };
 
     if (rows > 0) {
-      for (int tile = ta; tile < min(tb, tiles - 1); ++tile) {  // cache tiles of this piece
+      for (int tile = ta; tile < min(tb, segment_cache_tiles(tiles)); ++tile) {  // cache tiles
         const int k0 = tile * kTileKeys, k1 = min(k0 + kTileKeys, n);
         for (int c0 = k0; c0 < k1; c0 += kGenKC) {
           const int nk = min(kGenKC, k1 - c0);
@@ -215,9 +215,9 @@ attn_generic_kernel(AttnArgs a) {
         og[((size_t)(t0 + j) * a.Hq + g * G + i) * D + d] = from_f32<T>(acc[idx] / l_s[rho]);
       }
     } else {
-      float *P = a.ws.partials + (size_t)partial_slot(c, s0, W) * rows_max * (D + 2);
-      for (int idx = tid; idx < rows_max * (D + 2); idx += kGenThreads) {
-        const int rho = idx / (D + 2), d = idx % (D + 2);
+      float *P = a.ws.partials + (size_t)partial_slot(c, s0, W) * rows_max * part_stride(D);
+      for (int idx = tid; idx < rows_max * part_stride(D); idx += kGenThreads) {
+        const int rho = idx / part_stride(D), d = idx % part_stride(D);
         float val;
         if (rho < rows) val = (d < D) ? acc[rho * D + d] : (d == D ? m_s[rho] : l_s[rho]);
         else val = (d == D) ? -INFINITY : 0.f;
@@ -237,22 +237,22 @@ attn_generic_kernel(AttnArgs a) {
         for (int rho = warp; rho < rows; rho += NW) {
           float M = -INFINITY;
           for (int cc = c_first; cc <= c_last; ++cc) {
-            const float *Pp = a.ws.partials + (size_t)partial_slot(cc, s0, W) * rows_max * (D + 2);
-            M = fmaxf(M, __ldcg(Pp + rho * (D + 2) + D));
+            const float *Pp = a.ws.partials + (size_t)partial_slot(cc, s0, W) * rows_max * part_stride(D);
+            M = fmaxf(M, __ldcg(Pp + rho * part_stride(D) + D));
           }
           float Lsum = 0.f;
           for (int cc = c_first; cc <= c_last; ++cc) {
-            const float *Pp = a.ws.partials + (size_t)partial_slot(cc, s0, W) * rows_max * (D + 2);
-            const float mp = __ldcg(Pp + rho * (D + 2) + D);
-            if (mp != -INFINITY) Lsum += __ldcg(Pp + rho * (D + 2) + D + 1) * exp2f(mp - M);
+            const float *Pp = a.ws.partials + (size_t)partial_slot(cc, s0, W) * rows_max * part_stride(D);
+            const float mp = __ldcg(Pp + rho * part_stride(D) + D);
+            if (mp != -INFINITY) Lsum += __ldcg(Pp + rho * part_stride(D) + D + 1) * exp2f(mp - M);
           }
           const int j = rho / G, i = rho % G;
           for (int d = lane; d < D; d += 32) {
             float o = 0.f;
             for (int cc = c_first; cc <= c_last; ++cc) {
-              const float *Pp = a.ws.partials + (size_t)partial_slot(cc, s0, W) * rows_max * (D + 2);
-              const float mp = __ldcg(Pp + rho * (D + 2) + D);
-              if (mp != -INFINITY) o += __ldcg(Pp + rho * (D + 2) + d) * exp2f(mp - M);
+              const float *Pp = a.ws.partials + (size_t)partial_slot(cc, s0, W) * rows_max * part_stride(D);
+              const float mp = __ldcg(Pp + rho * part_stride(D) + D);
+              if (mp != -INFINITY) o += __ldcg(Pp + rho * part_stride(D) + d) * exp2f(mp - M);
             }
             og[((size_t)(t0 + j) * a.Hq + g * G + i) * D + d] = from_f32<T>(o / Lsum);
           }

@@ -44,27 +44,36 @@ namespace tc {
 
 constexpr int kPage = 64;                            // keys per page slot
 constexpr int kTK = 128;                             // keys per tile (two page slots)
-constexpr int kSlots = 6;                            // page slots per ring (three tile pairs)
-constexpr int kPairs = kSlots / 2;
-constexpr int kThreads = 192;
+// page slots per K ring and per V ring (even: a tile takes two).  K is released as soon as S has
+// been computed, V only after P.V, so V holds its slots longer.
+constexpr int kSlotsK = 6, kSlotsV = 6;
+constexpr int kPairsK = kSlotsK / 2, kPairsV = kSlotsV / 2;
+constexpr int kMaxSlots = 8;
+static_assert(kSlotsK % 2 == 0 && kSlotsV % 2 == 0 && kSlotsK <= kMaxSlots && kSlotsV <= kMaxSlots,
+              "slot counts");
+constexpr int kThreads = 224;
 constexpr int kSoftmaxThreads = 128;
 constexpr int kD = 128;
 constexpr int kNewRows = 16;                         // verify tokens per unit (K + 1 <= 16)
 constexpr uint32_t kSlotBytes = 64 * 128;            // 64 rows x 128 B: one d-half of a page
-constexpr uint32_t kRingBytes = kSlots * kSlotBytes; // one ring (K h0, K h1, V h0 or V h1)
-constexpr uint32_t kPageBytes = 4 * kSlotBytes;      // a full page: K and V, both d-halves
-constexpr uint32_t kNewBytes = 4 * kNewRows * 128;   // verify-token unit
-constexpr uint32_t kOffAux = 4 * kRingBytes;
+constexpr uint32_t kRingBytesK = kSlotsK * kSlotBytes;  // one K ring (d-half 0 or 1)
+constexpr uint32_t kRingBytesV = kSlotsV * kSlotBytes;  // one V ring
+constexpr uint32_t kHalfPageBytes = 2 * kSlotBytes;  // K (or V) of a page, both d-halves
+constexpr uint32_t kNewHalfBytes = 2 * kNewRows * 128;  // K (or V) of the verify-token unit
+constexpr uint32_t kOffAux = 2 * kRingBytesK + 2 * kRingBytesV;
 constexpr uint32_t kAuxBytes = 2048;
-constexpr uint32_t kOffScratch = kOffAux + kAuxBytes;
-constexpr uint32_t kScratchBytes = 128 * 16 * 4;     // epilogue: 128 lanes x 16 fp32
-constexpr uint32_t kSmemBytes = kOffScratch + kScratchBytes + 1024;  // + alignment slack
+// staging: the next piece's query rows (<= 64 x 256 B), then the epilogue's 128 x 32 fp32
+constexpr uint32_t kOffStage = kOffAux + kAuxBytes;
+constexpr uint32_t kStageBytes = 16384;
+constexpr uint32_t kSmemBytes = kOffStage + kStageBytes + 1024;  // + alignment slack
+constexpr int kPS = part_stride(kD);                 // floats per split-KV partial row
 
 // aux region layout (bytes)
-constexpr uint32_t kBarKvFull = 0, kBarKvEmpty = 64, kBarSFull = 128, kBarPFull = 144,
-                   kBarODone = 152, kBarQFull = 160, kBarQEmpty = 168, kBarOFree = 176;
-constexpr uint32_t kAuxTmem = 224, kAuxAbort = 228, kAuxLast = 232, kAuxPmax = 256,
-                   kAuxLsum = 256 + 2 * 128 * 4;
+constexpr uint32_t kBarKFull = 0, kBarVFull = 64, kBarKEmpty = 128, kBarVEmpty = 192,
+                   kBarSFull = 256, kBarPFull = 272, kBarODone = 280, kBarQFull = 288,
+                   kBarQEmpty = 296, kBarOFree = 304;
+constexpr uint32_t kAuxTmem = 320, kAuxAbort = 324, kAuxLast = 328, kAuxPmax = 512,
+                   kAuxLsum = 512 + 2 * 128 * 4;
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;
@@ -81,34 +90,23 @@ struct Meta {
   bool valid, last, newtile;                      // ncache: their 128-key tiles
 };
 
-// Serial validation of one piece [ta, tb) of a segment with `tiles` units; every role computes
-// it identically.
+// Metadata of one piece [ta, tb) of a segment with `tiles` units, from the plan's per-request
+// record (one 16-byte load); every role computes it identically.
 __device__ __forceinline__ Meta piece_meta(const AttnArgs &a, int r, int ta, int tb, int tiles,
                                            bool raise) {
   Meta m;
-  m.t0 = __ldg(a.q_offsets + r);
-  m.Q = __ldg(a.q_offsets + r + 1) - m.t0;
-  m.n = __ldg(a.kv_len + r);
-  bool ok = (m.Q >= 1 && m.Q <= a.K + 1 && m.t0 >= 0 && m.t0 + m.Q <= a.T_cap);
-  if (!ok && raise) raise_error(DSPARK_DERR_OFFSETS);
-  const bool okn =
-      (m.n >= 0 && (int64_t)(m.n + a.page_size - 1) / a.page_size <= a.max_pages);
+  const int4 rec = __ldg(a.ws.req + r);
+  m.t0 = rec.x;
+  m.Q = rec.y;
+  m.n = rec.z;
+  bool ok = rec.w != 0;
+  const bool okn = (int64_t)(m.n + a.page_size - 1) / a.page_size <= a.max_pages;
   if (ok && !okn && raise) raise_error(DSPARK_DERR_KV_LEN);
   ok = ok && okn;
-  if (ok) {
-    for (int j = 0; j < m.Q; ++j) {
-      if (__ldg(a.markers + 2 * (m.t0 + j)) != r ||
-          __ldg(a.markers + 2 * (m.t0 + j) + 1) != m.n + j) {
-        if (raise) raise_error(DSPARK_DERR_MARKER);
-        ok = false;
-        break;
-      }
-    }
-  }
   m.valid = ok;
   m.rows = ok ? a.G * m.Q : 0;
   m.C = m.rows <= 32 ? 4 : 2;
-  m.npages = ok ? max(0, min(tb, tiles - 1) - ta) : 0;
+  m.npages = ok ? max(0, min(tb, segment_cache_tiles(tiles)) - ta) : 0;
   m.ncache = (m.npages + 1) / 2;
   m.last = (tb == tiles);
   m.newtile = ok && m.last;
@@ -132,6 +130,39 @@ struct PieceIter {
     tb = min(tiles, ta + (u1 - u));
     u += tb - ta;
     return true;
+  }
+};
+
+// Walks the tiles of this CTA's pieces in order (pieces without tiles are skipped).  gt = global
+// tile index of the CTA, pq = index of the current piece among the pieces with tiles.
+struct TileCursor {
+  PieceIter it;
+  Meta m;
+  int r, g, ta, tb, tiles, s0, j;
+  uint32_t gt, pq;
+  bool ok;
+  __device__ __forceinline__ bool next_piece(const AttnArgs &a) {
+    while (it.next(a, r, g, ta, tb, tiles, s0)) {
+      m = piece_meta(a, r, ta, tb, tiles, false);
+      if (m.ntiles > 0) {
+        j = 0;
+        return true;
+      }
+    }
+    return false;
+  }
+  __device__ __forceinline__ void init(const AttnArgs &a) {
+    it.init(a);
+    gt = 0;
+    pq = 0;
+    ok = next_piece(a);
+  }
+  __device__ __forceinline__ void advance(const AttnArgs &a) {
+    ++gt;
+    if (++j == m.ntiles) {
+      ++pq;
+      ok = next_piece(a);
+    }
   }
 };
 
@@ -247,18 +278,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
   volatile int *abort_flag = reinterpret_cast<volatile int *>(gaux + kAuxAbort);
   float *pmax_buf = reinterpret_cast<float *>(gaux + kAuxPmax);
   float *lsum_buf = reinterpret_cast<float *>(gaux + kAuxLsum);
-  float *scratch = reinterpret_cast<float *>(gbase + kOffScratch);
+  const uint32_t stage = base + kOffStage;
   volatile int *s_last = reinterpret_cast<volatile int *>(gaux + kAuxLast);
   // ring r (0 = K d-half 0, 1 = K d-half 1, 2 = V d-half 0, 3 = V d-half 1), page slot s
-  auto ring = [&](int rg, uint32_t s) { return base + (uint32_t)rg * kRingBytes + s * kSlotBytes; };
+  auto ring = [&](int rg, uint32_t s) {
+    return base + (rg < 2 ? (uint32_t)rg * kRingBytesK
+                          : 2 * kRingBytesK + (uint32_t)(rg - 2) * kRingBytesV) + s * kSlotBytes;
+  };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   auto bar = [&](uint32_t off, int i) { return aux + off + 8u * (uint32_t)i; };
 
   if (tid == 0) {
-    for (int i = 0; i < kSlots; ++i) {
-      ptx::mbar_init(bar(kBarKvFull, i), 1);
-      ptx::mbar_init(bar(kBarKvEmpty, i), 1);
+    for (int i = 0; i < kSlotsK; ++i) {
+      ptx::mbar_init(bar(kBarKFull, i), 1);
+      ptx::mbar_init(bar(kBarKEmpty, i), 1);
+    }
+    for (int i = 0; i < kSlotsV; ++i) {
+      ptx::mbar_init(bar(kBarVFull, i), 1);
+      ptx::mbar_init(bar(kBarVEmpty, i), 1);
     }
     for (int i = 0; i < 2; ++i) ptx::mbar_init(bar(kBarSFull, i), 1);
     ptx::mbar_init(bar(kBarPFull, 0), kSoftmaxThreads);
@@ -288,117 +326,140 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
   it.init(a);
   int r, g, ta, tb, tiles, s0;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------------ TMA producer
+  if (warp == 4 || warp == 6) {
+    // ------------------------------------------------------------------ TMA producers
+    // warp 4 loads K, warp 6 loads V (a bulk L2 prefetch of later pages was tried and only
+    // lengthened the loads' latency).  Tile gt
+    // uses page slots 2(gt mod 3) and 2(gt mod 3) + 1 of both rings' families.
     if (lane == 0) {
-      uint32_t gs = 0;  // global page-slot counter (slot = gs % kSlots), always even per tile
-      int last_use[kSlots];  // latest slot use that was armed (TMA or empty arrive), -1 if none
+      const bool is_k = (warp == 4);
+      const uint32_t full0 = is_k ? kBarKFull : kBarVFull, empty0 = is_k ? kBarKEmpty : kBarVEmpty;
+      const int rg0 = is_k ? 0 : 2;
+      const CUtensorMap *nmap = is_k ? &tmap_kn : &tmap_vn;
+      const int nslots = is_k ? kSlotsK : kSlotsV;
+      int last_use[kMaxSlots];  // latest slot use that was armed (TMA or empty arrive), -1 if none
 #pragma unroll
-      for (int k = 0; k < kSlots; ++k) last_use[k] = -1;
-      auto wait_slot = [&](uint32_t sl) {
-        ptx::mbar_wait(bar(kBarKvEmpty, sl % kSlots), ((sl / kSlots) & 1) ^ 1, abort_flag);
-      };
-      while (it.next(a, r, g, ta, tb, tiles, s0)) {
-        const Meta m = piece_meta(a, r, ta, tb, tiles, false);
-        for (int j = 0; j < m.ntiles; ++j, gs += 2) {
-          for (int h = 0; h < 2; ++h) {   // the tile's two page slots
-            const uint32_t sl = gs + h, slot = sl % kSlots;
-            wait_slot(sl);
-            if (*abort_flag) continue;
-            const uint32_t fb = bar(kBarKvFull, slot);
-            const int pg = 2 * j + h;     // page of the piece in this slot
-            if (j < m.ncache && pg < m.npages) {
-              const int key0 = (ta + pg) * kPage;
-              const int page = __ldg(a.block_table + (size_t)r * a.max_pages + key0 / a.page_size);
-              int rowK = oob_row, rowV = oob_row;
-              if (page >= 0 && page < a.num_pages) {
-                rowK = ((page * 2) * a.Hkv + g) * a.page_size + key0 % a.page_size;
-                rowV = rowK + a.Hkv * a.page_size;
-              } else {
-                raise_error(DSPARK_DERR_PAGE);
-              }
-              ptx::mbar_arrive_expect_tx(fb, kPageBytes);
-              ptx::tma_load_2d(ring(0, slot), &tmap_kv, fb, 0, rowK);
-              ptx::tma_load_2d(ring(1, slot), &tmap_kv, fb, 64, rowK);
-              ptx::tma_load_2d(ring(2, slot), &tmap_kv, fb, 0, rowV);
-              ptx::tma_load_2d(ring(3, slot), &tmap_kv, fb, 64, rowV);
-            } else if (j == m.ncache && h == 0) {  // the verify tokens: 16 rows of KV head g
-              ptx::mbar_arrive_expect_tx(fb, kNewBytes);
-              ptx::tma_load_3d(ring(0, slot), &tmap_kn, fb, 0, g, m.t0);
-              ptx::tma_load_3d(ring(1, slot), &tmap_kn, fb, 64, g, m.t0);
-              ptx::tma_load_3d(ring(2, slot), &tmap_vn, fb, 0, g, m.t0);
-              ptx::tma_load_3d(ring(3, slot), &tmap_vn, fb, 64, g, m.t0);
-            } else {
-              ptx::mbar_arrive(fb);  // empty slot: completes its phase without data
+      for (int k = 0; k < kMaxSlots; ++k) last_use[k] = -1;
+      TileCursor tc;
+      tc.init(a);
+      while (tc.ok && !*abort_flag) {
+        const Meta &m = tc.m;
+        for (int h = 0; h < 2; ++h) {   // the tile's two page slots
+          const uint32_t sl = 2 * tc.gt + h, slot = sl % nslots;
+          ptx::mbar_wait(bar(empty0, slot), ((sl / nslots) & 1) ^ 1, abort_flag);
+          if (*abort_flag) break;
+          const uint32_t fb = bar(full0, slot);
+          const int pg = 2 * tc.j + h;     // page of the piece in this slot
+          if (tc.j < m.ncache && pg < m.npages) {
+            const int key0 = (tc.ta + pg) * kPage;
+            const int page = __ldg(a.block_table + (size_t)tc.r * a.max_pages + key0 / a.page_size);
+            int row = oob_row;
+            if (page >= 0 && page < a.num_pages) {
+              row = ((page * 2 + (is_k ? 0 : 1)) * a.Hkv + tc.g) * a.page_size + key0 % a.page_size;
+            } else if (is_k) {
+              raise_error(DSPARK_DERR_PAGE);
             }
-            last_use[slot] = (int)sl;
+            ptx::mbar_arrive_expect_tx(fb, kHalfPageBytes);
+            ptx::tma_load_2d(ring(rg0, slot), &tmap_kv, fb, 0, row);
+            ptx::tma_load_2d(ring(rg0 + 1, slot), &tmap_kv, fb, 64, row);
+          } else if (tc.j == m.ncache && h == 0) {  // the verify tokens: 16 rows of KV head g
+            ptx::mbar_arrive_expect_tx(fb, kNewHalfBytes);
+            ptx::tma_load_3d(ring(rg0, slot), nmap, fb, 0, tc.g, m.t0);
+            ptx::tma_load_3d(ring(rg0 + 1, slot), nmap, fb, 64, tc.g, m.t0);
+          } else {
+            ptx::mbar_arrive(fb);  // empty slot: completes its phase without data
           }
+          last_use[slot] = (int)sl;
         }
+        tc.advance(a);
       }
       // never leave the CTA with a bulk copy in flight: wait for the latest armed use of every
       // slot (its phase is the newest one the slot's barrier can complete)
       volatile int no_abort = 0;
-      for (int k = 0; k < kSlots; ++k)
+      for (int k = 0; k < nslots; ++k)
         if (last_use[k] >= 0)
-          ptx::mbar_wait(bar(kBarKvFull, k), ((uint32_t)last_use[k] / kSlots) & 1, &no_abort);
+          ptx::mbar_wait(bar(full0, k), ((uint32_t)last_use[k] / nslots) & 1, &no_abort);
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------------ MMA issuer
+    // Two cursors: S(js) for the next tile whose K has landed, P.V(jp) for the oldest tile whose
+    // P is written.  Whichever is ready is issued (P.V first), so a late K load never holds back
+    // the P.V of an earlier tile.  S runs at most one tile ahead of P.V (two S buffers: S(js)
+    // overwrites S(js - 2), which the softmax warps have read once P(js - 2) is published).
     if (lane == 0) {
-      uint32_t gt = 0, pq = 0;  // global tile counter, pieces with tiles
-      while (it.next(a, r, g, ta, tb, tiles, s0)) {
-        const Meta m = piece_meta(a, r, ta, tb, tiles, false);
-        if (m.ntiles == 0) continue;
-        ptx::mbar_wait(bar(kBarQFull, 0), pq & 1, abort_flag);
-        ptx::tc_fence_after();
-        auto issue_pv = [&](uint32_t gt_, int jj) {
-          if (jj == 0) {  // O of the previous piece has been read by its epilogue
-            ptx::mbar_wait(bar(kBarOFree, 0), (pq & 1) ^ 1, abort_flag);
+      TileCursor cs, cp;
+      cs.init(a);
+      cp.init(a);
+      long long idle_since = clock64();
+      while (cp.ok && !*abort_flag) {
+        bool progress = false;
+        if (cp.gt < cs.gt) {
+          const uint32_t pair = cp.gt % kPairsV, ph = (cp.gt / kPairsV) & 1;
+          if ((cp.j > 0 || ptx::mbar_test(bar(kBarOFree, 0), (cp.pq & 1) ^ 1)) &&
+              ptx::mbar_test(bar(kBarPFull, 0), cp.gt & 1) &&
+              ptx::mbar_test(bar(kBarVFull, 2 * pair), ph) &&
+              ptx::mbar_test(bar(kBarVFull, 2 * pair + 1), ph)) {
+            ptx::tc_fence_after();
+            const Meta &m = cp.m;
+            const int jj = cp.j;
+            const int ksteps = (jj < m.ncache) ? (min(kTK, m.npages * kPage - jj * kTK) / 16)
+                                               : kNewRows / 16;
+            // fully unrolled k-steps with compile-time descriptor offsets: the issue rate of
+            // tcgen05.mma drops several-fold when its operands are formed in a run-time loop
+            const uint64_t bd0 = ptx::smem_desc_sw128(ring(2, 2 * pair), kRingBytesV, 1024);
+            const uint32_t acc0 = jj > 0 ? 1u : 0u;
+            if (ksteps == kTK / 16) {
+#pragma unroll
+              for (int k = 0; k < kTK / 16; ++k)
+                ptx::mma_bf16_ts(tmem + kColO, tmem + kColP + k * 8, bd0 + (uint64_t)(k * 128),
+                                 kIdescPV, k > 0 ? 1u : acc0);
+            } else if (ksteps == kPage / 16) {
+#pragma unroll
+              for (int k = 0; k < kPage / 16; ++k)
+                ptx::mma_bf16_ts(tmem + kColO, tmem + kColP + k * 8, bd0 + (uint64_t)(k * 128),
+                                 kIdescPV, k > 0 ? 1u : acc0);
+            } else {
+              ptx::mma_bf16_ts(tmem + kColO, tmem + kColP, bd0, kIdescPV, acc0);
+            }
+            ptx::mma_commit(bar(kBarODone, 0));
+            ptx::mma_commit(bar(kBarVEmpty, 2 * pair));
+            ptx::mma_commit(bar(kBarVEmpty, 2 * pair + 1));
+            cp.advance(a);
+            progress = true;
           }
-          ptx::mbar_wait(bar(kBarPFull, 0), gt_ & 1, abort_flag);
-          ptx::tc_fence_after();
-          if (*abort_flag) return;
-          const uint32_t pair = gt_ % kPairs;
-          const int ksteps = (jj < m.ncache) ? (min(kTK, m.npages * kPage - jj * kTK) / 16)
-                                             : kNewRows / 16;
-          for (int k = 0; k < ksteps; ++k) {
-            const uint64_t bd =
-                ptx::smem_desc_sw128(ring(2, 2 * pair) + k * 2048, kRingBytes, 1024);
-            ptx::mma_bf16_ts(tmem + kColO, tmem + kColP + k * 8, bd, kIdescPV,
-                             (jj > 0 || k > 0) ? 1u : 0u);
-          }
-          ptx::mma_commit(bar(kBarODone, 0));
-          ptx::mma_commit(bar(kBarKvEmpty, 2 * pair));
-          ptx::mma_commit(bar(kBarKvEmpty, 2 * pair + 1));
-        };
-        for (int j = 0; j < m.ntiles; ++j) {
-          const uint32_t gt_ = gt + j;
-          const uint32_t pair = gt_ % kPairs;
-          const uint32_t ph = (gt_ / kPairs) & 1;
-          ptx::mbar_wait(bar(kBarKvFull, 2 * pair), ph, abort_flag);
-          ptx::mbar_wait(bar(kBarKvFull, 2 * pair + 1), ph, abort_flag);
-          ptx::tc_fence_after();
-          if (!*abort_flag) {
-            const uint32_t d_tmem = tmem + kColS + (gt_ & 1) * kTK;
+        }
+        if (!progress && cs.ok && cs.gt <= cp.gt + 1) {
+          const uint32_t pair = cs.gt % kPairsK, ph = (cs.gt / kPairsK) & 1;
+          if ((cs.j > 0 || ptx::mbar_test(bar(kBarQFull, 0), cs.pq & 1)) &&
+              ptx::mbar_test(bar(kBarKFull, 2 * pair), ph) &&
+              ptx::mbar_test(bar(kBarKFull, 2 * pair + 1), ph)) {
+            ptx::tc_fence_after();
+            const uint32_t d_tmem = tmem + kColS + (cs.gt & 1) * kTK;
 #pragma unroll
             for (int k = 0; k < kD / 16; ++k) {
               const uint32_t h = k >> 2, kk = k & 3;
               const uint64_t bd = ptx::smem_desc_sw128(ring(h, 2 * pair) + kk * 32, 16, 1024);
               ptx::mma_bf16_ts(d_tmem, tmem + kColQ + k * 8, bd, kIdescS, k > 0 ? 1u : 0u);
             }
-            ptx::mma_commit(bar(kBarSFull, gt_ & 1));
+            ptx::mma_commit(bar(kBarSFull, cs.gt & 1));
+            ptx::mma_commit(bar(kBarKEmpty, 2 * pair));
+            ptx::mma_commit(bar(kBarKEmpty, 2 * pair + 1));
             // the piece's last S read of Q: the next piece may stage its queries
-            if (j == m.ntiles - 1) ptx::mma_commit(bar(kBarQEmpty, 0));
+            if (cs.j == cs.m.ntiles - 1) ptx::mma_commit(bar(kBarQEmpty, 0));
+            cs.advance(a);
+            progress = true;
           }
-          if (j > 0) issue_pv(gt_ - 1, j - 1);
         }
-        issue_pv(gt + m.ntiles - 1, m.ntiles - 1);
-        gt += m.ntiles;
-        ++pq;
+        if (progress) {
+          idle_since = clock64();
+        } else if (clock64() - idle_since > ptx::kWaitLimitCycles) {
+          *abort_flag = 1;
+          raise_error(DSPARK_DERR_TIMEOUT);
+        }
       }
-      if (gt > 0 && !*abort_flag) {  // every MMA of this CTA has completed before TMEM is released
+      if (cp.gt > 0 && !*abort_flag) {  // every MMA of this CTA has completed before TMEM is released
         volatile int no_abort = 0;
-        ptx::mbar_wait(bar(kBarODone, 0), (gt - 1) & 1, &no_abort);
+        ptx::mbar_wait(bar(kBarODone, 0), (cp.gt - 1) & 1, &no_abort);
       }
     }
   } else {
@@ -410,27 +471,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
     const int G = a.G;
     uint32_t gt = 0, qidx = 0;
 
-    // A piece's queries, replicated per copy, into this lane's Q columns once the previous
-    // piece's last S MMA no longer reads them (inactive lanes get zeros).
-    auto stage_q = [&](const Meta &mq, int gq) {
-      const int rpcq = 128 / mq.C, rq = t % rpcq;
+    // A piece's query rows (row rq = j * G + i: token j, query head g * G + i) into the staging
+    // area with asynchronous 16-byte copies, chunk c of row rq at chunk slot c ^ (rq & 7) so the
+    // lane-per-row reads of q_commit spread over the banks.
+    auto q_prefetch = [&](const Meta &mq, int gq) {
+      for (int idx = t; idx < mq.rows * 16; idx += kSoftmaxThreads) {
+        const int rq = idx >> 4, c = idx & 15;
+        const int j = rq / G, i = rq % G;
+        ptx::cp_async16(stage + rq * 256 + ((c ^ (rq & 7)) << 4),
+                        qg + ((size_t)(mq.t0 + j) * a.Hq + gq * G + i) * kD + c * 8);
+      }
+      ptx::cp_async_commit();
+    };
+    // Staged rows into this lane's Q columns (replicated per copy; inactive lanes get zeros) once
+    // the previous piece's last S MMA no longer reads them.
+    auto q_commit = [&](const Meta &mq) {
+      ptx::cp_async_wait_all();
+      ptx::named_bar_sync(1, kSoftmaxThreads);  // every thread's copies have landed
+      const int rq = t % (128 / mq.C);
       ptx::mbar_wait(bar(kBarQEmpty, 0), (qidx & 1) ^ 1, abort_flag);
       ptx::tc_fence_after();
-      uint32_t w[32];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        if (rq < mq.rows) {
-          const int j = rq / G, i = rq % G;
-          const uint4 *src = reinterpret_cast<const uint4 *>(
-              qg + ((size_t)(mq.t0 + j) * a.Hq + gq * G + i) * kD + h * 64);
+        uint32_t w[32];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 v = __ldg(src + c);
-            w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) w[c] = 0u;
+        for (int c = 0; c < 8; ++c) {
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (rq < mq.rows) v = ptx::ld_shared_v4(stage + rq * 256 + (((h * 8 + c) ^ (rq & 7)) << 4));
+          w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
         }
         ptx::tmem_st<32>(tmem + lane_base + kColQ + h * 32, w);
       }
@@ -438,15 +506,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar(kBarQFull, 0));
       ++qidx;
+      ptx::named_bar_sync(1, kSoftmaxThreads);  // every lane has read the staging area
     };
 
     bool have = it.next(a, r, g, ta, tb, tiles, s0);
     Meta m;
     if (have) {
       m = piece_meta(a, r, ta, tb, tiles, t == 0);
-      if (m.ntiles > 0) stage_q(m, g);
+      if (m.ntiles > 0) {
+        q_prefetch(m, g);
+        q_commit(m);
+      }
     }
     while (have) {
+      // look one piece ahead: its metadata now, its queries on their way into the staging area
+      // while this piece's tiles stream
+      int r2, g2, ta2, tb2, tiles2, s02;
+      const bool have2 = it.next(a, r2, g2, ta2, tb2, tiles2, s02);
+      Meta m2;
+      if (have2) {
+        m2 = piece_meta(a, r2, ta2, tb2, tiles2, t == 0);
+        if (m2.ntiles > 0) q_prefetch(m2, g2);
+      }
+
       const int rpc = 128 / m.C;         // lanes per copy
       const int copy = t / rpc, rho = t % rpc;
       const bool active = m.valid && rho < m.rows;
@@ -481,8 +563,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
         // P = 0 times V stays 0 (the MMA reads whole 16-key steps of valid pages)
         const int vrows = cache_tile ? min(kTK, (vk + kPage - 1) / kPage * kPage) : kNewRows;
         if (vk < vrows) {
-          const uint32_t pair = gt_ % kPairs;
-          ptx::mbar_wait(bar(kBarKvFull, 2 * pair + vk / kPage), (gt_ / kPairs) & 1, abort_flag);
+          const uint32_t pair = gt_ % kPairsV;
+          ptx::mbar_wait(bar(kBarVFull, 2 * pair + vk / kPage), (gt_ / kPairsV) & 1, abort_flag);
           for (int idx = t; idx < (vrows - vk) * 16; idx += kSoftmaxThreads) {
             const uint32_t row = vk + idx / 16, half = (idx % 16) / 8, c = idx % 8;
             st_shared_v4(ring(2 + half, 2 * pair) + row * 128 + c * 16, 0u, 0u, 0u, 0u);
@@ -494,16 +576,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
         ptx::mbar_arrive(bar(kBarPFull, 0));
       }
 
-      // stage the next piece's queries now, so the MMAs of the next piece overlap this epilogue
-      int r2, g2, ta2, tb2, tiles2, s02;
-      const bool have2 = it.next(a, r2, g2, ta2, tb2, tiles2, s02);
-      Meta m2;
-      if (have2) {
-        m2 = piece_meta(a, r2, ta2, tb2, tiles2, t == 0);
-        if (m2.ntiles > 0) stage_q(m2, g2);
-      }
+      // the next piece's queries into tensor memory, so its S MMAs overlap this epilogue
+      if (have2 && m2.ntiles > 0) q_commit(m2);
 
       // ---------------------------------------------------------------- epilogue
+      // Each copy holds a partial O over its own keys.  Four rounds of 32 columns: every lane
+      // puts its columns into the staging area, then lane (copy, rho) sums the copies of row rho
+      // for its 32 / C columns of the round and writes them (bf16 output, or the fp32 partial of
+      // a split segment).
       lsum_buf[t] = sm.l_part;
       if (m.ntiles > 0) {
         ptx::mbar_wait(bar(kBarODone, 0), (gt + m.ntiles - 1) & 1, abort_flag);
@@ -512,8 +592,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       ptx::named_bar_sync(2, kSoftmaxThreads);
       const bool whole = (ta == 0 && tb == tiles);
       const int W = it.W;
-      float *part = a.ws.partials +
-                    (size_t)partial_slot(blockIdx.x, s0, W) * a.rows_max * (kD + 2);
+      float *part = a.ws.partials + (size_t)partial_slot(blockIdx.x, s0, W) * a.rows_max * kPS;
       if (m.ntiles > 0) {
         float l = 0.f;
         for (int cc = 0; cc < m.C; ++cc) l += lsum_buf[rho + cc * rpc];
@@ -521,50 +600,70 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
         const int j = rho / G, i = rho % G;
         const size_t orow = ((size_t)(m.t0 + j) * a.Hq + g * G + i) * kD;
         const uint32_t o_taddr = tmem + lane_base + kColO;
+        const int nc = 32 / m.C;  // columns of a round this lane finishes (8 or 16)
 #pragma unroll 1
-        for (int c16 = 0; c16 < 8; ++c16) {
-          float o[16];
-          ptx::tmem_ld16(o_taddr + c16 * 16, o);  // this copy's partial O
+        for (int c32 = 0; c32 < 4; ++c32) {
+          float o[32];
+          ptx::tmem_ld32(o_taddr + c32 * 32, o);
           ptx::tmem_wait_ld();
-          // sum the copies' partial O rows through shared memory
-          float4 *sv = reinterpret_cast<float4 *>(scratch + t * 16);
+          if (c32 == 3) {  // O fully read: the next piece's P.V may overwrite it
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(bar(kBarOFree, 0));
+          }
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sv[e] = make_float4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+          for (int k = 0; k < 8; ++k)
+            st_shared_v4(stage + t * 128 + ((k ^ (t & 7)) << 4), __float_as_uint(o[4 * k]),
+                         __float_as_uint(o[4 * k + 1]), __float_as_uint(o[4 * k + 2]),
+                         __float_as_uint(o[4 * k + 3]));
           ptx::named_bar_sync(2, kSoftmaxThreads);
-          if (copy == 0) {
-            for (int cc = 1; cc < m.C; ++cc) {
-              const float4 *sv2 = reinterpret_cast<const float4 *>(scratch + (rho + cc * rpc) * 16);
+          if (active) {
+            float acc[16];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float4 x = sv2[e];
-                o[4 * e] += x.x; o[4 * e + 1] += x.y; o[4 * e + 2] += x.z; o[4 * e + 3] += x.w;
+            for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+            const int k0 = copy * (nc / 4);   // first float4 chunk of this lane's columns
+            for (int cc = 0; cc < m.C; ++cc) {
+              const int row = rho + cc * rpc;
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                if (k < nc / 4) {
+                  const uint4 v = ptx::ld_shared_v4(stage + row * 128 + (((k0 + k) ^ (row & 7)) << 4));
+                  acc[4 * k] += __uint_as_float(v.x);
+                  acc[4 * k + 1] += __uint_as_float(v.y);
+                  acc[4 * k + 2] += __uint_as_float(v.z);
+                  acc[4 * k + 3] += __uint_as_float(v.w);
+                }
               }
             }
-          }
-          ptx::named_bar_sync(2, kSoftmaxThreads);
-          if (active && copy == 0) {
+            const int col0 = c32 * 32 + copy * nc;
             if (whole) {
-              uint32_t w8[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) w8[e] = ptx::pack_bf16x2(o[2 * e] * inv, o[2 * e + 1] * inv);
-              uint4 *dst = reinterpret_cast<uint4 *>(og + orow + c16 * 16);
-              dst[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-              dst[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+              for (int k = 0; k < 4; ++k) {
+                if (k < nc / 4) {
+                  uint2 w2;
+                  w2.x = ptx::pack_bf16x2(acc[4 * k] * inv, acc[4 * k + 1] * inv);
+                  w2.y = ptx::pack_bf16x2(acc[4 * k + 2] * inv, acc[4 * k + 3] * inv);
+                  *reinterpret_cast<uint2 *>(og + orow + col0 + 4 * k) = w2;
+                }
+              }
             } else {
-              // rows are 130 floats apart: 8-byte aligned, so float2 stores
-              float2 *dst = reinterpret_cast<float2 *>(part + (size_t)rho * (kD + 2) + c16 * 16);
+              float4 *dst = reinterpret_cast<float4 *>(part + (size_t)rho * kPS + col0);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) dst[e] = make_float2(o[2 * e], o[2 * e + 1]);
+              for (int k = 0; k < 4; ++k)
+                if (k < nc / 4)
+                  dst[k] = make_float4(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3]);
             }
           }
+          ptx::named_bar_sync(2, kSoftmaxThreads);  // before the next round reuses the staging
         }
         if (active && copy == 0 && !whole) {
-          part[(size_t)rho * (kD + 2) + kD] = sm.m_run;
-          part[(size_t)rho * (kD + 2) + kD + 1] = l;
+          part[(size_t)rho * kPS + kD] = sm.m_run;
+          part[(size_t)rho * kPS + kD + 1] = l;
         }
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(bar(kBarOFree, 0));
         gt += m.ntiles;
+      } else if (!whole) {
+        // a piece holding only tail units of its segment: a partial without keys
+        for (int idx = t; idx < m.rows * kPS; idx += kSoftmaxThreads)
+          part[idx] = (idx % kPS == kD) ? -INFINITY : 0.f;
       }
 
       if (!whole) {  // split segment: publish the partial, the last piece merges
@@ -579,50 +678,71 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
         if (*s_last) {
           __threadfence();
           const int c_first = s0 / W, c_last = (s0 + tiles - 1) / W;
-          const size_t pstride = (size_t)a.rows_max * (kD + 2);
+          const size_t pstride = (size_t)a.rows_max * kPS;
           const float *P0 = a.ws.partials;
-          // per row: merged maximum and 1 / merged sum (threads t < rows)
+          // per row: merged maximum and 1 / merged sum (threads t < rows); the loads of four
+          // pieces are in flight at once
           float *Ms = pmax_buf, *Li = lsum_buf;
           if (t < m.rows) {
-            float M = -INFINITY;
-            for (int cc = c_first; cc <= c_last; ++cc)
-              M = fmaxf(M, __ldcg(P0 + (size_t)partial_slot(cc, s0, W) * pstride +
-                                  (size_t)t * (kD + 2) + kD));
-            float L = 0.f;
-            for (int cc = c_first; cc <= c_last; ++cc) {
-              const float *Pp = P0 + (size_t)partial_slot(cc, s0, W) * pstride + (size_t)t * (kD + 2);
-              const float mp = __ldcg(Pp + kD);
-              if (mp != -INFINITY) L += __ldcg(Pp + kD + 1) * ex2(mp - M);
+            float M = -INFINITY, L = 0.f;
+            for (int c4 = c_first; c4 <= c_last; c4 += 4) {
+              float mp[4], lp[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int cc = min(c4 + k, c_last);
+                const float *Pp = P0 + (size_t)partial_slot(cc, s0, W) * pstride + (size_t)t * kPS;
+                mp[k] = __ldcg(Pp + kD);
+                lp[k] = __ldcg(Pp + kD + 1);
+              }
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                if (c4 + k <= c_last && mp[k] != -INFINITY) {
+                  const float Mn = fmaxf(M, mp[k]);
+                  L = L * ex2(M - Mn) + lp[k] * ex2(mp[k] - Mn);
+                  M = Mn;
+                }
+              }
             }
             Ms[t] = M;
             Li[t] = 1.f / L;
           }
           ptx::named_bar_sync(2, kSoftmaxThreads);
-          // thread t owns head-dim column t; 8 rows at a time keep 8 x pieces loads in flight
-          const int d = t;
-          for (int row0 = 0; row0 < m.rows; row0 += 8) {
-            float o[8];
+          // items (row, float4 column): this thread's items of a group of 8 accumulate piece by
+          // piece, each piece's loads for the group in flight together
+          const int nitems = m.rows * (kD / 4);
+          for (int it0 = t; it0 < nitems; it0 += 8 * kSoftmaxThreads) {
+            float4 acc[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) o[k] = 0.f;
+            for (int k = 0; k < 8; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int cc = c_first; cc <= c_last; ++cc) {
               const float *Pp = P0 + (size_t)partial_slot(cc, s0, W) * pstride;
 #pragma unroll
               for (int k = 0; k < 8; ++k) {
-                const int row = row0 + k;
-                if (row < m.rows) {
-                  const float mp = __ldcg(Pp + (size_t)row * (kD + 2) + kD);
-                  const float v = __ldcg(Pp + (size_t)row * (kD + 2) + d);
-                  if (mp != -INFINITY) o[k] = fmaf(v, ex2(mp - Ms[row]), o[k]);
+                const int item = it0 + k * kSoftmaxThreads;
+                if (item < nitems) {
+                  const int row = item / (kD / 4), d4 = item % (kD / 4);
+                  const float mp = __ldcg(Pp + (size_t)row * kPS + kD);
+                  const float4 v = __ldcg(reinterpret_cast<const float4 *>(Pp + (size_t)row * kPS) + d4);
+                  const float wgt = (mp == -INFINITY) ? 0.f : ex2(mp - Ms[row]);
+                  acc[k].x = fmaf(v.x, wgt, acc[k].x);
+                  acc[k].y = fmaf(v.y, wgt, acc[k].y);
+                  acc[k].z = fmaf(v.z, wgt, acc[k].z);
+                  acc[k].w = fmaf(v.w, wgt, acc[k].w);
                 }
               }
             }
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-              const int row = row0 + k;
-              if (row < m.rows) {
+              const int item = it0 + k * kSoftmaxThreads;
+              if (item < nitems) {
+                const int row = item / (kD / 4), d4 = item % (kD / 4);
                 const int jj = row / G, ii = row % G;
-                og[((size_t)(m.t0 + jj) * a.Hq + g * G + ii) * kD + d] =
-                    __float2bfloat16_rn(o[k] * Li[row]);
+                const float li = Li[row];
+                uint2 w2;
+                w2.x = ptx::pack_bf16x2(acc[k].x * li, acc[k].y * li);
+                w2.y = ptx::pack_bf16x2(acc[k].z * li, acc[k].w * li);
+                *reinterpret_cast<uint2 *>(og + ((size_t)(m.t0 + jj) * a.Hq + g * G + ii) * kD +
+                                           d4 * 4) = w2;
               }
             }
           }
@@ -638,7 +758,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       }
     }
   }
-
   __syncthreads();
   if (warp == 5) {
     ptx::tc_fence_after();

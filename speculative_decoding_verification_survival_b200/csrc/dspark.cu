@@ -147,10 +147,11 @@ size_t dspark_verify_attn_workspace_bytes(int R, int Hq, int Hkv, int D, int K) 
   return attn_ws_layout(R, Hkv, (Hq / Hkv) * (K + 1), D, ctas, nullptr, nullptr);
 }
 
-int dspark_verify_attn_plan(const int32_t *kv_len, int R, int Hq, int Hkv, int D, int K, void *ws,
-                            size_t ws_bytes, dspark_stream_t stream) {
-  if (!kv_len || R < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || D < 8 || D > 256 || D % 8 ||
-      K < 1 || K > DSPARK_MAX_K)
+int dspark_verify_attn_plan(const int32_t *kv_len, const int32_t *q_offsets,
+                            const int32_t *markers, int R, int T_cap, int Hq, int Hkv, int D,
+                            int K, void *ws, size_t ws_bytes, dspark_stream_t stream) {
+  if (!kv_len || !q_offsets || !markers || R < 1 || T_cap < R || Hkv < 1 || Hq < Hkv ||
+      Hq % Hkv != 0 || D < 8 || D > 256 || D % 8 || K < 1 || K > DSPARK_MAX_K)
     return DSPARK_EINVAL;
   if (!ws || !aligned16(ws)) return DSPARK_EWORKSPACE;
   const int ctas = max_attn_ctas();
@@ -158,8 +159,8 @@ int dspark_verify_attn_plan(const int32_t *kv_len, int R, int Hq, int Hkv, int D
   const int rows_max = (Hq / Hkv) * (K + 1);
   AttnWs w;
   if (ws_bytes < attn_ws_layout(R, Hkv, rows_max, D, ctas, &w, ws)) return DSPARK_EWORKSPACE;
-  attn_plan_kernel<<<1, 1024, 0, reinterpret_cast<cudaStream_t>(stream)>>>(kv_len, R, Hkv,
-                                                                           rows_max, D, w);
+  attn_plan_kernel<<<1, 1024, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      kv_len, q_offsets, markers, R, T_cap, K, Hkv, rows_max, D, w);
   return launch_status();
 }
 

@@ -54,7 +54,7 @@ _SIGS = {
     "dspark_version": ([], _i),
     "dspark_schedule": ([_p, _i, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p], _i),
     "dspark_verify_attn_workspace_bytes": ([_i, _i, _i, _i, _i], _sz),
-    "dspark_verify_attn_plan": ([_p, _i, _i, _i, _i, _i, _p, _sz, _p], _i),
+    "dspark_verify_attn_plan": ([_p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _sz, _p], _i),
     "dspark_verify_attn": ([_p, _p, _p, _p, _i64, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i,
                             _i, _i, _f, _p, _p, _sz, _p], _i),
     "dspark_accept_workspace_bytes": ([_i, _i, _i], _sz),
@@ -134,10 +134,12 @@ def dspark_verify_attn_workspace_bytes(R, Hq, Hkv, D, K) -> int:
     return int(_lib.dspark_verify_attn_workspace_bytes(R, Hq, Hkv, D, K))
 
 
-def dspark_verify_attn_plan(kv_len, R, Hq, Hkv, D, K, ws, stream=None):
-    _check(kv_len, torch.int32, "kv_len")
-    _call("dspark_verify_attn_plan", _ptr(kv_len), R, Hq, Hkv, D, K, _ptr(ws), ws.numel(),
-          _stream(stream))
+def dspark_verify_attn_plan(kv_len, q_offsets, markers, R, Hq, Hkv, D, K, ws, stream=None):
+    """kv_len int32 [R]; q_offsets int32 [R + 1]; markers int32 [T_cap][2]."""
+    for t, n in ((kv_len, "kv_len"), (q_offsets, "q_offsets"), (markers, "markers")):
+        _check(t, torch.int32, n)
+    _call("dspark_verify_attn_plan", _ptr(kv_len), _ptr(q_offsets), _ptr(markers), R,
+          markers.shape[0], Hq, Hkv, D, K, _ptr(ws), ws.numel(), _stream(stream))
 
 
 def dspark_verify_attn(q, k_new, v_new, kv_pages, block_table, kv_len, markers, q_offsets, K,

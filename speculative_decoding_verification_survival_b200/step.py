@@ -43,8 +43,8 @@ class VerifyStep:
                            self.q_offsets, self.markers, self.T, self.objective, stream)
 
     def plan(self, kv_len, stream=None):
-        _d.dspark_verify_attn_plan(kv_len, self.R, self.Hq, self.Hkv, self.D, self.K,
-                                   self.attn_ws, stream)
+        _d.dspark_verify_attn_plan(kv_len, self.q_offsets, self.markers, self.R, self.Hq,
+                                   self.Hkv, self.D, self.K, self.attn_ws, stream)
 
     def attention(self, q, k_new, v_new, kv_pages, block_table, kv_len, out, stream=None):
         _d.dspark_verify_attn(q, k_new, v_new, kv_pages, block_table, kv_len, self.markers,
