@@ -63,10 +63,15 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            # start timing only once the sampler is producing (nvidia-smi takes a while to start)
+            t_end = time.time() + 10.0
+            while not self.lines and time.time() < t_end and self.proc.poll() is None:
+                time.sleep(0.02)
+            self.lines.clear()
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
@@ -102,6 +107,33 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch, from an ncu
+# capture of the bench's own command (the summary under profiles/ gives the command), keyed by the
+# SHA-1 of the kernel sources the capture ran; any change to those sources voids the figure.
+NCU_TRAFFIC = {
+    # profiles/attn_tc_kernel_qwen3-4b-64req_full.md: 630.775808 MB read + 8.089344 MB written
+    "qwen3-4b-64req": ("c318ecbae831d9905849f59e91a7eff0c60e7b6c", 638865152),
+}
+
+
+def kernel_source_hash():
+    import hashlib
+    d = os.path.join(ROOT, "speculative_decoding_verification_survival_b200", "csrc")
+    h = hashlib.sha1()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(d, name), "rb") as fh:
+                h.update(name.encode() + b"\0" + fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload):
+    rec = NCU_TRAFFIC.get(workload)
+    if rec is None or rec[0] != kernel_source_hash():
+        return None
+    return rec[1]
 
 
 def attn_bytes(kv_len, verify_len, cfg):
@@ -306,7 +338,7 @@ def cpu_baseline(cfg, max_seconds: float = 20.0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="dspark", choices=["dspark", "reference"])
     ap.add_argument("--workload", default="qwen3-4b-64req", choices=sorted(CONFIGS))
@@ -385,7 +417,8 @@ def main():
             step_hbm_gbs=step_gbs, step_frac_of_8tbs=step_gbs / 8000.0,
             step_frac_of_measured=step_gbs / peak,
             roofline=dict(bound="hbm", kernel="dspark_verify_attn", achieved=achieved, peak=peak,
-                          unit="GB/s", frac=achieved / peak, traffic=None,
+                          unit="GB/s", frac=achieved / peak,
+                          traffic=measured_traffic(cfg.name),
                           peak_source=peak_kind,
                           bytes_per_launch=res["attn_bytes"], ms_per_launch=attn_ms),
             e2e=dict(value=L_tot / (e2e_ms * 1e-3), unit=UNIT,
