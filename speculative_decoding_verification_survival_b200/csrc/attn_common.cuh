@@ -24,7 +24,8 @@ constexpr int kMaxCtasPerSm = 4;
 
 struct AttnPlanHeader {
   int R, Hkv, rows_max, D;
-  int tile_keys, pad0, pad1, pad2;
+  int tile_keys, total;  // total = units of the whole batch
+  int tc_ctas, tc_W;     // the tensor-core kernel's grid and units per CTA
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -37,6 +38,7 @@ struct AttnWs {
   int *tile_prefix;  // [R + 1]: first unit of request r (units of all its Hkv segments)
   int *counters;     // [R * Hkv] arrival counters of split segments (kept at zero between calls)
   int4 *req;         // [R]: per request {t0, Q, kv_len, schedule valid} written by the plan
+  int4 *cta_start;   // [max_ctas]: first segment of tensor-core CTA c {r, g, s0, units}, r < 0: none
   float *partials;   // [2 * max_ctas][rows_max][part_stride(D)]: acc[D], m, l per row
 };
 
@@ -47,6 +49,7 @@ __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, i
   const size_t o_pre = off;                off += align256((size_t)(R + 1) * sizeof(int));
   const size_t o_cnt = off;                off += align256((size_t)R * Hkv * sizeof(int));
   const size_t o_req = off;                off += align256((size_t)R * sizeof(int4));
+  const size_t o_cst = off;                off += align256((size_t)max_ctas * sizeof(int4));
   const size_t o_par = off;
   off += align256((size_t)2 * max_ctas * rows_max * part_stride(D) * sizeof(float));
   if (ws) {
@@ -55,6 +58,7 @@ __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, i
     ws->tile_prefix = reinterpret_cast<int *>(b + o_pre);
     ws->counters = reinterpret_cast<int *>(b + o_cnt);
     ws->req = reinterpret_cast<int4 *>(b + o_req);
+    ws->cta_start = reinterpret_cast<int4 *>(b + o_cst);
     ws->partials = reinterpret_cast<float *>(b + o_par);
   }
   return off;
@@ -79,10 +83,15 @@ __host__ __device__ inline int segment_cache_tiles(int units) { return units - k
 // carries the marker (r, kv_len + j) — the layout the scheduler's flattening step produces).
 // A malformed request raises its error bit here, once per step, and is skipped by the
 // attention calls that use this plan.
+__device__ __forceinline__ void find_segment(const int *__restrict__ tile_prefix, int R, int Hkv,
+                                             int u, int &r, int &g, int &tiles, int &seg_start);
+
+// It also records where each of the tensor-core kernel's `tc_ctas` CTAs starts (its first
+// segment), so that kernel walks segments in order without searching.
 __global__ void __launch_bounds__(1024)
 attn_plan_kernel(const int32_t *__restrict__ kv_len, const int32_t *__restrict__ q_offsets,
                  const int32_t *__restrict__ markers, int R, int T_cap, int K, int Hkv,
-                 int rows_max, int D, AttnWs ws) {
+                 int rows_max, int D, int tc_ctas, AttnWs ws) {
   __shared__ int warp_tot[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = (R + blockDim.x - 1) / blockDim.x;
@@ -136,12 +145,27 @@ attn_plan_kernel(const int32_t *__restrict__ kv_len, const int32_t *__restrict__
     }
     ws.req[r] = make_int4(t0, Q, n, ok ? 1 : 0);
   }
+  __syncthreads();  // tile_prefix complete (global writes of this block)
+  const int total = ws.tile_prefix[R];
+  const int W = (total + tc_ctas - 1) / tc_ctas;
+  for (int c = tid; c < tc_ctas; c += blockDim.x) {
+    int4 st = make_int4(-1, 0, 0, 0);
+    if (c * W < total) {
+      int r, g, tiles, s0;
+      find_segment(ws.tile_prefix, R, Hkv, c * W, r, g, tiles, s0);
+      st = make_int4(r, g, s0, tiles);
+    }
+    ws.cta_start[c] = st;
+  }
   if (tid == 0) {
     ws.hdr->R = R;
     ws.hdr->Hkv = Hkv;
     ws.hdr->rows_max = rows_max;
     ws.hdr->D = D;
     ws.hdr->tile_keys = kTileKeys;
+    ws.hdr->total = total;
+    ws.hdr->tc_ctas = tc_ctas;
+    ws.hdr->tc_W = W;
   }
 }
 
@@ -154,17 +178,18 @@ struct SegPiece {
   bool first_of_cta;
 };
 
-// Locate the segment containing global unit u (binary search over requests).
+// Locate the segment containing global unit u (binary search over requests).  Plain loads: the
+// plan kernel calls it on a prefix it has just written.
 __device__ __forceinline__ void find_segment(const int *__restrict__ tile_prefix, int R, int Hkv,
                                              int u, int &r, int &g, int &tiles, int &seg_start) {
   int lo = 0, hi = R - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(tile_prefix + mid) <= u) lo = mid; else hi = mid - 1;
+    if (tile_prefix[mid] <= u) lo = mid; else hi = mid - 1;
   }
   r = lo;
-  const int base = __ldg(tile_prefix + r);
-  tiles = (__ldg(tile_prefix + r + 1) - base) / Hkv;
+  const int base = tile_prefix[r];
+  tiles = (tile_prefix[r + 1] - base) / Hkv;
   g = (u - base) / tiles;
   seg_start = base + g * tiles;
 }

@@ -114,21 +114,42 @@ __device__ __forceinline__ Meta piece_meta(const AttnArgs &a, int r, int ta, int
   return m;
 }
 
+// This CTA's contiguous range of units [u, u1) as pieces (one per segment it touches), walking
+// the segments in order from the CTA's start record written by the plan.
 struct PieceIter {
   int u, u1, W;
+  int r, g, tiles, s0;  // current segment
   __device__ __forceinline__ void init(const AttnArgs &a) {
-    const int total = __ldg(a.ws.tile_prefix + a.R);
-    W = (total + gridDim.x - 1) / gridDim.x;
+    const int total = __ldg(&a.ws.hdr->total);
+    const int ctas = __ldg(&a.ws.hdr->tc_ctas);
+    if (ctas == (int)gridDim.x) {
+      W = __ldg(&a.ws.hdr->tc_W);
+      const int4 st = __ldg(a.ws.cta_start + blockIdx.x);
+      r = st.x; g = st.y; s0 = st.z; tiles = st.w;
+    } else {  // a grid the plan did not prepare for: search for the first segment
+      W = (total + gridDim.x - 1) / gridDim.x;
+      r = -1;
+      if ((int64_t)blockIdx.x * W < total)
+        find_segment(a.ws.tile_prefix, a.R, a.Hkv, blockIdx.x * W, r, g, tiles, s0);
+    }
     u = blockIdx.x * W;
-    u1 = min(u + W, total);
+    u1 = (r < 0) ? u : min(u + W, total);
   }
-  __device__ __forceinline__ bool next(const AttnArgs &a, int &r, int &g, int &ta, int &tb,
-                                       int &tiles, int &s0) {
+  __device__ __forceinline__ bool next(const AttnArgs &a, int &r_, int &g_, int &ta, int &tb,
+                                       int &tiles_, int &s0_) {
     if (u >= u1) return false;
-    find_segment(a.ws.tile_prefix, a.R, a.Hkv, u, r, g, tiles, s0);
+    r_ = r; g_ = g; tiles_ = tiles; s0_ = s0;
     ta = u - s0;
-    tb = min(tiles, ta + (u1 - u));
-    u += tb - ta;
+    tb = min(tiles, u1 - s0);
+    u = s0 + tb;
+    if (tb == tiles && u < u1) {  // on to the next segment: (r, g + 1) or (r + 1, 0)
+      s0 += tiles;
+      if (++g == a.Hkv) {
+        g = 0;
+        ++r;
+        tiles = (__ldg(a.ws.tile_prefix + r + 1) - __ldg(a.ws.tile_prefix + r)) / a.Hkv;
+      }
+    }
     return true;
   }
 };
@@ -321,6 +342,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(gaux + kAuxTmem);
+  // Launched with programmatic stream serialisation: the prologue above overlaps the previous
+  // kernel's tail; nothing written by an earlier kernel is read before this wait.  The next
+  // launch may then start its own prologue as soon as SMs free up.
+  ptx::grid_dependency_wait();
+  ptx::grid_launch_dependents();
 
   PieceIter it;
   it.init(a);

@@ -160,7 +160,7 @@ int dspark_verify_attn_plan(const int32_t *kv_len, const int32_t *q_offsets,
   AttnWs w;
   if (ws_bytes < attn_ws_layout(R, Hkv, rows_max, D, ctas, &w, ws)) return DSPARK_EWORKSPACE;
   attn_plan_kernel<<<1, 1024, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      kv_len, q_offsets, markers, R, T_cap, K, Hkv, rows_max, D, w);
+      kv_len, q_offsets, markers, R, T_cap, K, Hkv, rows_max, D, sm_count(), w);
   return launch_status();
 }
 
@@ -210,8 +210,20 @@ int dspark_verify_attn(const void *q, const void *k_new, const void *v_new, cons
     if (cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)tc::kSmemBytes) != cudaSuccess)
       return DSPARK_ECUDA;
-    tc::attn_tc_kernel<<<sms, tc::kThreads, tc::kSmemBytes, s>>>(map, map_kn, map_vn, a,
-                                                                (int)kv_rows);
+    // programmatic stream serialisation: the kernel's prologue may overlap the previous kernel
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sms);
+    cfg.blockDim = dim3(tc::kThreads);
+    cfg.dynamicSmemBytes = tc::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel, map, map_kn, map_vn, a, (int)kv_rows) !=
+        cudaSuccess)
+      return DSPARK_ECUDA;
     return launch_status();
   }
   const size_t smem = attn_generic_smem_bytes(rows_max, D);
