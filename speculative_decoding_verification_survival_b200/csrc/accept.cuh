@@ -11,11 +11,12 @@
 //                          (r, k) with k < verify_len[r] unless greedy).  One streaming pass:
 //                          per-thread running max with float32 exp2 terms accumulated into
 //                          float64 sums (rescaled when the running max rises), then a block
-//                          merge -> (m, Z = sum exp((z - m)/tau), argmax with lowest index).
-//   accept_finalize_kernel one CTA per request: the accept chain (thread 0), then the
-//                          correction / bonus draw by inverse CDF over one row pair: pass 1
-//                          sums the weights per 2048-element chunk (float64), the threshold
-//                          u * Z picks the chunk, pass 2 re-reads that chunk and scans it.
+//                          merge -> (m, Z = sum exp((z - m)/tau); greedy: argmax, lowest index).
+//   accept_finalize_kernel one CTA per request: all draft positions tested at once, the accepted
+//                          prefix ends at the first failure; then the correction / bonus draw
+//                          by inverse CDF over one row pair: pass 1 sums the weights per
+//                          2048-element chunk (float64), the threshold u * Z picks the chunk,
+//                          pass 2 re-reads that chunk and scans it.
 #pragma once
 
 #include "common.cuh"
@@ -23,11 +24,12 @@
 namespace dspark {
 
 constexpr int kAccThreads = 256;
-constexpr int kAccChunk = kAccThreads * 8;
+constexpr int kAccWarps = kAccThreads / 32;
+constexpr int kAccChunk = kAccThreads * 8;  // elements per chunk of the inverse-CDF scan
 
 struct RowStats {
   float m;      // row maximum
-  int argmax;   // lowest index attaining m
+  int argmax;   // lowest index attaining m (greedy verification only)
   double Z;     // sum_v exp2((z_v - m) * c), c = log2(e) / tau
 };
 
@@ -35,14 +37,31 @@ __host__ __device__ inline size_t accept_ws_bytes(int R, int K, int T_cap) {
   return ((size_t)T_cap + (size_t)R * K) * sizeof(RowStats);
 }
 
+// Dynamic shared memory of the finalize kernel: per-warp partial sums of every chunk, then the
+// chunk sums and two scalars.
+__host__ __device__ inline size_t accept_finalize_smem(int V) {
+  const size_t nch = ((size_t)V + kAccChunk - 1) / kAccChunk;
+  return ((size_t)kAccWarps * nch + nch + 2) * sizeof(double);
+}
+
 template <typename T>
 __device__ __forceinline__ float ld1(const T *p) { return to_f32(__ldg(p)); }
 
-template <typename T>
+// 2^x with the SFU (relative error about 2^-22; results below 2^-126 flush to zero).
+__device__ __forceinline__ float exp2_sfu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// One CTA per scheduled logit row: one streaming pass with 16-byte loads, 32 elements per thread
+// and step; the running maximum rescales the float64 sum only when it rises.  GREEDY rows only
+// need the maximum and its lowest index.
+template <typename T, bool GREEDY>
 __global__ void __launch_bounds__(kAccThreads)
 accept_stats_kernel(const T *__restrict__ target, const T *__restrict__ draft, int V, int R, int K,
                     int T_cap, const int32_t *__restrict__ verify_len,
-                    const int32_t *__restrict__ q_offsets, float c, int greedy,
+                    const int32_t *__restrict__ q_offsets, float c,
                     RowStats *__restrict__ stats) {
   const int b = blockIdx.x;
   const T *row;
@@ -51,7 +70,7 @@ accept_stats_kernel(const T *__restrict__ target, const T *__restrict__ draft, i
     if (b >= Tn) return;
     row = target + (size_t)b * V;
   } else {
-    if (greedy) return;
+    if (GREEDY) return;
     const int i = b - T_cap, r = i / K, k = i % K;
     const int L = __ldg(verify_len + r);
     if (k >= L) return;
@@ -61,76 +80,95 @@ accept_stats_kernel(const T *__restrict__ target, const T *__restrict__ draft, i
   float m = -INFINITY;
   double Z = 0.0;
   int amax = 0x7fffffff;
-  const bool vec = ((reinterpret_cast<uintptr_t>(row) & 15) == 0) && (V % 8 == 0) &&
-                   (sizeof(T) == 2 || (reinterpret_cast<uintptr_t>(row) & 31) == 0);
-  auto consume = [&](const float (&x)[8], int base, int cnt) {
-    float mx = -INFINITY;
-    int ix = 0x7fffffff;
+  // x[u][e] is element base[u] + e; groups are visited in index order
+  auto consume = [&](const float (&x)[4][8], const int (&base)[4]) {
+    if (GREEDY) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      if (e < cnt && x[e] > mx) { mx = x[e]; ix = base + e; }
-    }
-    if (mx > m) {
-      if (!greedy && m != -INFINITY) Z *= exp2((double)(m - mx) * (double)c);
-      m = mx;
-      amax = ix;
-    }
-    if (!greedy && m != -INFINITY) {
-      float s = 0.f;
+      for (int u = 0; u < 4; ++u)
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if (e < cnt) s += exp2f((x[e] - m) * c);
-      Z += (double)s;
+        for (int e = 0; e < 8; ++e)
+          if (x[u][e] > m) { m = x[u][e]; amax = base[u] + e; }
+    } else {
+      float lm = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) lm = fmaxf(lm, x[u][e]);
+      if (lm > m) {
+        if (m != -INFINITY) Z *= exp2((double)(m - lm) * (double)c);
+        m = lm;
+      }
+      if (m != -INFINITY) {
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            s0 += exp2_sfu((x[u][e] - m) * c);
+            s1 += exp2_sfu((x[u][e + 1] - m) * c);
+          }
+        Z += (double)(s0 + s1);
+      }
     }
   };
+  const bool vec = ((reinterpret_cast<uintptr_t>(row) & 15) == 0) && (V % 8 == 0) &&
+                   (sizeof(T) == 2 || (reinterpret_cast<uintptr_t>(row) & 31) == 0);
   if (vec) {
     const int nv = V / 8;
-    int v8 = tid;
-    for (; v8 + 3 * kAccThreads < nv; v8 += 4 * kAccThreads) {
+    for (int v8 = tid; v8 < nv; v8 += 4 * kAccThreads) {
       float x[4][8];
+      int base[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) load8(row + (size_t)(v8 + u * kAccThreads) * 8, x[u]);
+      for (int u = 0; u < 4; ++u) {
+        const int g = v8 + u * kAccThreads;
+        base[u] = g * 8;
+        if (g < nv) {
+          load8(row + (size_t)g * 8, x[u]);
+        } else {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) consume(x[u], (v8 + u * kAccThreads) * 8, 8);
-    }
-    for (; v8 < nv; v8 += kAccThreads) {
-      float x[8];
-      load8(row + (size_t)v8 * 8, x);
-      consume(x, v8 * 8, 8);
+          for (int e = 0; e < 8; ++e) x[u][e] = -INFINITY;
+        }
+      }
+      consume(x, base);
     }
   } else {
-    for (int base = tid * 8; base < V; base += kAccThreads * 8) {
-      float x[8];
-      const int cnt = min(8, V - base);
+    for (int b0 = tid * 8; b0 < V; b0 += 4 * kAccThreads * 8) {
+      float x[4][8];
+      int base[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = (e < cnt) ? ld1(row + base + e) : -INFINITY;
-      consume(x, base, cnt);
+      for (int u = 0; u < 4; ++u) {
+        base[u] = b0 + u * kAccThreads * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          x[u][e] = (base[u] + e < V) ? ld1(row + base[u] + e) : -INFINITY;
+      }
+      consume(x, base);
     }
   }
   // block merge
-  __shared__ float sm_m[kAccThreads / 32];
-  __shared__ int sm_i[kAccThreads / 32];
-  __shared__ double sm_z[kAccThreads / 32];
+  __shared__ float sm_m[kAccWarps];
+  __shared__ int sm_i[kAccWarps];
+  __shared__ double sm_z[kAccWarps];
   const int lane = tid & 31, warp = tid >> 5;
-  float wm = warp_max(m);
+  const float wm = warp_max(m);
   int wi = (m == wm) ? amax : 0x7fffffff;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) wi = min(wi, __shfl_xor_sync(0xffffffffu, wi, o));
   if (lane == 0) { sm_m[warp] = wm; sm_i[warp] = wi; }
   __syncthreads();
   float M = sm_m[0];
-  for (int w = 1; w < kAccThreads / 32; ++w) M = fmaxf(M, sm_m[w]);
+  for (int w = 1; w < kAccWarps; ++w) M = fmaxf(M, sm_m[w]);
   int I = 0x7fffffff;
-  for (int w = 0; w < kAccThreads / 32; ++w)
+  for (int w = 0; w < kAccWarps; ++w)
     if (sm_m[w] == M) I = min(I, sm_i[w]);
-  double z = (!greedy && m != -INFINITY && M != -INFINITY) ? Z * exp2((double)(m - M) * (double)c)
-                                                          : 0.0;
+  double z = (!GREEDY && m != -INFINITY && M != -INFINITY) ? Z * exp2((double)(m - M) * (double)c)
+                                                           : 0.0;
   z = warp_sum(z);
   if (lane == 0) sm_z[warp] = z;
   __syncthreads();
   if (tid == 0) {
     double Zt = 0.0;
-    for (int w = 0; w < kAccThreads / 32; ++w) Zt += sm_z[w];
+    for (int w = 0; w < kAccWarps; ++w) Zt += sm_z[w];
     if (!(M > -INFINITY && M < INFINITY)) raise_error(DSPARK_DERR_LOGITS);
     RowStats st;
     st.m = M;
@@ -140,46 +178,74 @@ accept_stats_kernel(const T *__restrict__ target, const T *__restrict__ draft, i
   }
 }
 
+// Per-element weights are float32 (their exp2 is float32 anyway, relative error ~2^-22); the
+// sums over the vocabulary are float64 (groups of 8 summed in float32 first).  Float64 is a slow
+// pipe on this part, so it is kept out of the per-element work.
 template <typename T>
 struct RowPair {
   const T *t;  // target row
   const T *d;  // draft row (residual only)
   float mt, md;
-  double invZt, invZd;
+  float invZt, invZd;
   float c;
-  bool residual;
-  __device__ __forceinline__ double weight(float zt, float zd) const {
-    const double pt = (double)exp2f((zt - mt) * c) * invZt;
+  bool residual, vec;
+  __device__ __forceinline__ float weight(float zt, float zd) const {
+    const float pt = exp2_sfu((zt - mt) * c) * invZt;
     if (!residual) return pt;
-    const double qd = (double)exp2f((zd - md) * c) * invZd;
-    return fmax(0.0, pt - qd);
+    return fmaxf(0.f, pt - exp2_sfu((zd - md) * c) * invZd);
   }
 };
 
-// Sum of the weights of elements [base, base + 8) of the row pair (float64, in index order).
-template <typename T>
-__device__ __forceinline__ double weights8(const RowPair<T> &rp, int base, int V, double (&w)[8]) {
-  double s = 0.0;
+// Eight consecutive logits as raw bits (one 16-byte load for bf16, two for f32), so that a
+// step's loads are all issued before any of them is converted.
+template <typename T> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> { uint4 a; };
+template <> struct Raw8<float> { float4 a, b; };
+__device__ __forceinline__ void load_raw8(const __nv_bfloat16 *p, Raw8<__nv_bfloat16> &r) {
+  r.a = __ldg(reinterpret_cast<const uint4 *>(p));
+}
+__device__ __forceinline__ void load_raw8(const float *p, Raw8<float> &r) {
+  r.a = __ldg(reinterpret_cast<const float4 *>(p));
+  r.b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+}
+__device__ __forceinline__ void cvt8(const Raw8<__nv_bfloat16> &r, float (&v)[8]) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&r.a);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int v = base + e;
-    double x = 0.0;
-    if (v < V) x = rp.weight(ld1(rp.t + v), rp.residual ? ld1(rp.d + v) : 0.f);
-    w[e] = x;
-    s += x;
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
   }
-  return s;
+}
+__device__ __forceinline__ void cvt8(const Raw8<float> &r, float (&v)[8]) {
+  v[0] = r.a.x; v[1] = r.a.y; v[2] = r.a.z; v[3] = r.a.w;
+  v[4] = r.b.x; v[5] = r.b.y; v[6] = r.b.z; v[7] = r.b.w;
 }
 
-__device__ __forceinline__ double block_sum_f64(double x, double *sm) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  x = warp_sum(x);
-  if (lane == 0) sm[warp] = x;
-  __syncthreads();
-  double t = 0.0;
-  for (int w = 0; w < kAccThreads / 32; ++w) t += sm[w];
-  __syncthreads();
-  return t;
+// Logits [base, base + 8) of the row pair, element by element (any alignment; -inf past V).
+template <typename T>
+__device__ __forceinline__ void load_pair8_scalar(const RowPair<T> &rp, int base, int V,
+                                                  float (&xt)[8], float (&xd)[8]) {
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const bool in = base + e < V;
+    xt[e] = in ? ld1(rp.t + base + e) : -INFINITY;
+    xd[e] = (in && rp.residual) ? ld1(rp.d + base + e) : 0.f;
+  }
+}
+
+// Weights of elements [base, base + 8) (0 past the end) and their sum in index order.
+template <typename T>
+__device__ __forceinline__ double weights8(const RowPair<T> &rp, int base, int V,
+                                           const float (&xt)[8], const float (&xd)[8],
+                                           float (&w)[8]) {
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    w[e] = (base + e < V) ? rp.weight(xt[e], xd[e]) : 0.f;
+    s += w[e];
+  }
+  return (double)s;
 }
 
 __device__ __forceinline__ double block_excl_scan_f64_acc(double x, double *sm) {
@@ -198,18 +264,58 @@ __device__ __forceinline__ double block_excl_scan_f64_acc(double x, double *sm) 
   return off + incl - x;
 }
 
-// Inverse-CDF draw over a row pair: smallest v with C(v) > u * C(V-1).
+// Inverse-CDF draw over a row pair: smallest v with C(v) > u * C(V-1).  Pass 1 streams the row
+// (four chunks per step with every load of the step issued before any is used, per-warp partial
+// sums in shared memory, no barrier inside the loop); the threshold picks a chunk; pass 2
+// re-reads that chunk and scans it in index order.
 template <typename T>
-__device__ int draw_inverse_cdf(const RowPair<T> &rp, int V, float u, double *chunk_sum,
-                                double *sm) {
+__device__ int draw_inverse_cdf(const RowPair<T> &rp, int V, float u, double *fsm, double *sm) {
   __shared__ int s_pick;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nch = (V + kAccChunk - 1) / kAccChunk;
-  for (int ch = 0; ch < nch; ++ch) {
-    double w[8];
-    const double s = weights8(rp, ch * kAccChunk + tid * 8, V, w);
-    const double tot = block_sum_f64(s, sm);
-    if (tid == 0) chunk_sum[ch] = tot;
+  double *part = fsm;                         // [kAccWarps][nch]
+  double *chunk_sum = fsm + kAccWarps * nch;  // [nch + 2]
+  constexpr int kU = 4;
+  for (int ch0 = 0; ch0 < nch; ch0 += kU) {
+    float xt[kU][8], xd[kU][8];
+    if (rp.vec) {  // V % 8 == 0, rows aligned: a group is either wholly inside or past the end
+      Raw8<T> rt[kU], rd[kU];
+#pragma unroll
+      for (int k = 0; k < kU; ++k) {
+        const int base = (ch0 + k) * kAccChunk + tid * 8;
+        const int b = base < V ? base : 0;  // in-bounds address; values past V are masked below
+        load_raw8(rp.t + b, rt[k]);
+        if (rp.residual) load_raw8(rp.d + b, rd[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < kU; ++k) {
+        cvt8(rt[k], xt[k]);
+        if (rp.residual) {
+          cvt8(rd[k], xd[k]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xd[k][e] = 0.f;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < kU; ++k)
+        load_pair8_scalar(rp, (ch0 + k) * kAccChunk + tid * 8, V, xt[k], xd[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < kU; ++k) {
+      if (ch0 + k < nch) {
+        float w[8];
+        const double s = warp_sum(weights8(rp, (ch0 + k) * kAccChunk + tid * 8, V, xt[k], xd[k], w));
+        if (lane == 0) part[warp * nch + ch0 + k] = s;
+      }
+    }
+  }
+  __syncthreads();
+  for (int ch = tid; ch < nch; ch += kAccThreads) {
+    double t = 0.0;
+    for (int w = 0; w < kAccWarps; ++w) t += part[w * nch + ch];
+    chunk_sum[ch] = t;
   }
   __syncthreads();
   if (tid == 0) {
@@ -236,9 +342,11 @@ __device__ int draw_inverse_cdf(const RowPair<T> &rp, int V, float u, double *ch
   const int pick = s_pick;
   if (pick < 0) return -1;  // no mass anywhere
   const double thr = chunk_sum[nch], base = chunk_sum[nch + 1];
-  double w[8];
   const int b0 = pick * kAccChunk + tid * 8;
-  const double s = weights8(rp, b0, V, w);
+  float xt[8], xd[8];
+  load_pair8_scalar(rp, b0, V, xt, xd);
+  float w[8];
+  const double s = weights8(rp, b0, V, xt, xd, w);
   const double ex = block_excl_scan_f64_acc(s, sm);
   __shared__ int s_found, s_lastpos;
   if (tid == 0) { s_found = 0x7fffffff; s_lastpos = -1; }
@@ -247,8 +355,8 @@ __device__ int draw_inverse_cdf(const RowPair<T> &rp, int V, float u, double *ch
   double C = base + ex;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    C += w[e];
-    if (w[e] > 0.0) {
+    C += (double)w[e];
+    if (w[e] > 0.f) {
       lastpos = b0 + e;
       if (base >= 0.0 && C > thr && found == 0x7fffffff) found = b0 + e;
     }
@@ -259,82 +367,90 @@ __device__ int draw_inverse_cdf(const RowPair<T> &rp, int V, float u, double *ch
   return (s_found != 0x7fffffff) ? s_found : s_lastpos;
 }
 
-template <typename T>
+// One CTA per request: every draft position's test at once (one thread each), the accepted
+// prefix ending at the first failure, then the correction / bonus token.
+template <typename T, bool GREEDY>
 __global__ void __launch_bounds__(kAccThreads)
 accept_finalize_kernel(const T *__restrict__ target, const T *__restrict__ draft, int V, int R,
                        int K, int T_cap, const int32_t *__restrict__ draft_tokens,
                        const int32_t *__restrict__ verify_len,
                        const int32_t *__restrict__ q_offsets, const float *__restrict__ u_acc,
-                       const float *__restrict__ u_res, float c, int greedy,
+                       const float *__restrict__ u_res, float c,
                        const RowStats *__restrict__ stats, int32_t *__restrict__ accepted_len,
                        int32_t *__restrict__ out_tokens, int32_t *__restrict__ n_out) {
-  extern __shared__ double chunk_sum[];  // [nch + 2]
-  __shared__ double sm[kAccThreads / 32];
-  __shared__ int s_a, s_ok;
+  extern __shared__ double fsm[];
+  __shared__ double sm[kAccWarps];
+  __shared__ int s_fail;
   const int r = blockIdx.x, tid = threadIdx.x;
   const int L = __ldg(verify_len + r);
   const int t0 = __ldg(q_offsets + r), t1 = __ldg(q_offsets + r + 1);
+  const bool len_ok = L >= 0 && L <= K;
+  const bool ok = len_ok && t1 - t0 == L + 1 && t0 >= 0 && t1 <= T_cap;
   if (tid == 0) {
-    int ok = 1;
-    if (L < 0 || L > K) { raise_error(DSPARK_DERR_VERIFY_LEN); ok = 0; }
-    else if (t1 - t0 != L + 1 || t0 < 0 || t1 > T_cap) { raise_error(DSPARK_DERR_OFFSETS); ok = 0; }
-    int a = 0;
-    if (ok) {
-      for (; a < L; ++a) {
-        const int x = __ldg(draft_tokens + (size_t)r * K + a);
-        if (x < 0 || x >= V) { raise_error(DSPARK_DERR_TOKEN); break; }
-        const RowStats st = stats[t0 + a];
-        if (greedy) {
-          if (x != st.argmax) break;
-        } else {
-          const RowStats sd = stats[T_cap + r * K + a];
-          const float zt = ld1(target + (size_t)(t0 + a) * V + x);
-          const float zd = ld1(draft + ((size_t)r * K + a) * V + x);
-          const double p = (double)exp2f((zt - st.m) * c) / st.Z;
-          const double q = (double)exp2f((zd - sd.m) * c) / sd.Z;
-          const double ratio = (q > 0.0) ? p / q : (p > 0.0 ? INFINITY : 0.0);
-          const double thr = fmin(1.0, ratio);
-          if (!((double)__ldg(u_acc + (size_t)r * K + a) < thr)) break;
-        }
-      }
-    }
-    s_a = a;
-    s_ok = ok;
+    if (!len_ok) raise_error(DSPARK_DERR_VERIFY_LEN);
+    else if (!ok) raise_error(DSPARK_DERR_OFFSETS);
+    s_fail = ok ? L : 0;
   }
   __syncthreads();
-  const int a = s_a;
-  if (!s_ok) {
+  if (!ok) {
     for (int j = tid; j <= K; j += kAccThreads) out_tokens[(size_t)r * (K + 1) + j] = -1;
     if (tid == 0) { accepted_len[r] = 0; n_out[r] = 0; }
     return;
   }
+  bool bad = false;
+  if (tid < L) {
+    const int x = __ldg(draft_tokens + (size_t)r * K + tid);
+    bad = x < 0 || x >= V;
+    bool fail = bad;
+    if (!bad) {
+      const RowStats st = stats[t0 + tid];
+      if (GREEDY) {
+        fail = x != st.argmax;
+      } else {
+        const RowStats sd = stats[T_cap + r * K + tid];
+        const float zt = ld1(target + (size_t)(t0 + tid) * V + x);
+        const float zd = ld1(draft + ((size_t)r * K + tid) * V + x);
+        const double p = (double)exp2_sfu((zt - st.m) * c) / st.Z;
+        const double q = (double)exp2_sfu((zd - sd.m) * c) / sd.Z;
+        const double ratio = (q > 0.0) ? p / q : (p > 0.0 ? INFINITY : 0.0);
+        fail = !((double)__ldg(u_acc + (size_t)r * K + tid) < fmin(1.0, ratio));
+      }
+    }
+    if (fail) atomicMin(&s_fail, tid);
+  }
+  __syncthreads();
+  const int a = s_fail;
+  if (tid == a && bad) raise_error(DSPARK_DERR_TOKEN);  // the token the chain stopped at
   int corr;
-  if (greedy) {
+  if (GREEDY) {
     corr = stats[t0 + a].argmax;
   } else {
     RowPair<T> rp;
     const RowStats st = stats[t0 + a];
     rp.t = target + (size_t)(t0 + a) * V;
     rp.mt = st.m;
-    rp.invZt = 1.0 / st.Z;
+    rp.invZt = (float)(1.0 / st.Z);
     rp.c = c;
     rp.residual = a < L;
     if (rp.residual) {
       const RowStats sd = stats[T_cap + r * K + a];
       rp.d = draft + ((size_t)r * K + a) * V;
       rp.md = sd.m;
-      rp.invZd = 1.0 / sd.Z;
+      rp.invZd = (float)(1.0 / sd.Z);
     } else {
       rp.d = nullptr;
       rp.md = 0.f;
-      rp.invZd = 0.0;
+      rp.invZd = 0.f;
     }
+    const size_t align = sizeof(T) == 2 ? 15 : 31;
+    rp.vec = (V % 8 == 0) && ((reinterpret_cast<uintptr_t>(rp.t) & align) == 0) &&
+             (!rp.residual || (reinterpret_cast<uintptr_t>(rp.d) & align) == 0);
     const float u = __ldg(u_res + (size_t)r * (K + 1) + a);
-    corr = draw_inverse_cdf(rp, V, u, chunk_sum, sm);
+    corr = draw_inverse_cdf(rp, V, u, fsm, sm);
     if (corr < 0 && rp.residual) {  // residual empty in floating point: draw from p instead
       rp.residual = false;
       __syncthreads();
-      corr = draw_inverse_cdf(rp, V, u, chunk_sum, sm);
+      corr = draw_inverse_cdf(rp, V, u, fsm, sm);
     }
   }
   for (int j = tid; j <= K; j += kAccThreads) {

@@ -267,25 +267,27 @@ int dspark_accept(const void *target_logits, const void *draft_logits, int dtype
   RowStats *st = static_cast<RowStats *>(ws);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int nrows = T_cap + R * K;
-  const int nch = (V + kAccChunk - 1) / kAccChunk;
-  const size_t fin_smem = (size_t)(nch + 2) * sizeof(double);
+  const size_t fin_smem = accept_finalize_smem(V);
   if (fin_smem > 227 * 1024) return DSPARK_EUNSUPPORTED;
   auto run = [&](auto tag) -> int {
     using T = decltype(tag);
     const T *tl = static_cast<const T *>(target_logits);
     const T *dl = static_cast<const T *>(draft_logits);
-    accept_stats_kernel<T><<<nrows, kAccThreads, 0, s>>>(tl, dl, V, R, K, T_cap, verify_len,
-                                                         q_offsets, c, greedy ? 1 : 0, st);
-    if (cudaGetLastError() != cudaSuccess) return DSPARK_ECUDA;
-    if (fin_smem > 48 * 1024 &&
-        cudaFuncSetAttribute(accept_finalize_kernel<T>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)fin_smem) != cudaSuccess)
-      return DSPARK_ECUDA;
-    accept_finalize_kernel<T><<<R, kAccThreads, fin_smem, s>>>(
-        tl, dl, V, R, K, T_cap, draft_tokens, verify_len, q_offsets, u_acc, u_res, c,
-        greedy ? 1 : 0, st, accepted_len, out_tokens, n_out);
-    return launch_status();
+    auto launch = [&](auto stats_kernel, auto fin_kernel) -> int {
+      stats_kernel<<<nrows, kAccThreads, 0, s>>>(tl, dl, V, R, K, T_cap, verify_len, q_offsets,
+                                                 c, st);
+      if (cudaGetLastError() != cudaSuccess) return DSPARK_ECUDA;
+      if (fin_smem > 48 * 1024 &&
+          cudaFuncSetAttribute(fin_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)fin_smem) != cudaSuccess)
+        return DSPARK_ECUDA;
+      fin_kernel<<<R, kAccThreads, fin_smem, s>>>(tl, dl, V, R, K, T_cap, draft_tokens,
+                                                  verify_len, q_offsets, u_acc, u_res, c, st,
+                                                  accepted_len, out_tokens, n_out);
+      return launch_status();
+    };
+    if (greedy) return launch(accept_stats_kernel<T, true>, accept_finalize_kernel<T, true>);
+    return launch(accept_stats_kernel<T, false>, accept_finalize_kernel<T, false>);
   };
   if (dtype == DSPARK_BF16) return run(__nv_bfloat16());
   return run(float());
