@@ -335,6 +335,21 @@ def cpu_baseline(cfg, max_seconds: float = 20.0):
     return float(L.sum()) / step_s, desc, 1, step_s
 
 
+def reduce_replicas(ms_step, attn_ms, e2e_ms, L_sum, acc_sum, R, world, device):
+    """Combine independent replicas: times are the max over ranks (the job waits for the
+    slowest), token and request counts are summed (every rank verifies its own batch)."""
+    vec = torch.tensor([ms_step, attn_ms, e2e_ms, L_sum, acc_sum, R], dtype=torch.float64,
+                       device=device)
+    mx, sm = vec, vec
+    if world > 1:
+        mx = vec.clone()
+        torch.distributed.all_reduce(mx, op=torch.distributed.ReduceOp.MAX)
+        sm = vec.clone()
+        torch.distributed.all_reduce(sm, op=torch.distributed.ReduceOp.SUM)
+    return dict(ms_step=float(mx[0]), attn_ms=float(mx[1]), e2e_ms=float(mx[2]),
+                L_tot=float(sm[3]), acc_tot=float(sm[4]), R_tot=float(sm[5]))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -380,22 +395,11 @@ def main():
     torch.cuda.set_device(device)
     cfg, res = run_dspark(args, rank, world, device)
 
-    L_sum, acc_sum = int(res["L"].sum()), int(res["acc"].sum())
     R = cfg.R
-    ms_step = res["ms_total"] / args.steps
-    e2e_ms = res["e2e"]["ms"]
-    vec = torch.tensor([ms_step, res["attn_ms"], e2e_ms, L_sum, acc_sum, R], dtype=torch.float64,
-                       device=device)
-    if world > 1:
-        mx = vec.clone()
-        torch.distributed.all_reduce(mx, op=torch.distributed.ReduceOp.MAX)
-        sm = vec.clone()
-        torch.distributed.all_reduce(sm, op=torch.distributed.ReduceOp.SUM)
-        ms_step, attn_ms, e2e_ms = float(mx[0]), float(mx[1]), float(mx[2])
-        L_tot, acc_tot, R_tot = float(sm[3]), float(sm[4]), float(sm[5])
-    else:
-        attn_ms = res["attn_ms"]
-        L_tot, acc_tot, R_tot = float(L_sum), float(acc_sum), float(R)
+    agg = reduce_replicas(res["ms_total"] / args.steps, res["attn_ms"], res["e2e"]["ms"],
+                          int(res["L"].sum()), int(res["acc"].sum()), R, world, device)
+    ms_step, attn_ms, e2e_ms = agg["ms_step"], agg["attn_ms"], agg["e2e_ms"]
+    L_tot, acc_tot, R_tot = agg["L_tot"], agg["acc_tot"], agg["R_tot"]
 
     if rank == 0:
         peak, peak_kind = measured_peaks()
