@@ -10,6 +10,7 @@
  *                          request's paged KV cache and its own earlier verify tokens
  *   dspark_accept          exact acceptance rule, longest accepted prefix, residual / bonus
  *                          resampling (or greedy verification)
+ *   dspark_kv_commit       the kept tokens' K/V into the paged cache (after acceptance)
  *
  * Conventions shared by every entry point:
  *   - Every pointer argument is DEVICE memory owned by the caller, unless stated otherwise.
@@ -73,7 +74,8 @@ enum dspark_device_error {
   DSPARK_DERR_VERIFY_LEN = 1 << 6,  /* verify_len outside [0, K] */
   DSPARK_DERR_TOKEN = 1 << 7,       /* a draft token outside [0, V) */
   DSPARK_DERR_LOGITS = 1 << 8,      /* a logit row whose maximum is not finite */
-  DSPARK_DERR_TIMEOUT = 1 << 9      /* a bounded in-kernel wait expired; results undefined */
+  DSPARK_DERR_TIMEOUT = 1 << 9,     /* a bounded in-kernel wait expired; results undefined */
+  DSPARK_DERR_ACCEPTED = 1 << 10    /* an accepted length outside [0, verify_len] */
 };
 
 #define DSPARK_CONF_LAG 2             /* rounds between producing and consuming confidences */
@@ -244,6 +246,37 @@ int dspark_accept_noalloc(const void *target_logits, const void *draft_logits, i
                           const float *u_acc, const float *u_res, float temperature,
                           int32_t *accepted_len, int32_t *out_tokens, int32_t *n_out,
                           dspark_stream_t stream);
+
+/*
+ * dspark_kv_commit — the kept verify rows of every request join its paged KV cache.
+ *
+ * Defined by [P1 opening section: drafts the target confirms are adopted, "猜对了就采纳"] and
+ * [P2 §一: the verified tokens are kept].  After dspark_accept, request r keeps its verify tokens
+ * j = 0 .. accepted_len[r]: token 0 sits at position kv_len[r] (the previous round's last
+ * emitted token, whose K/V this verify pass computed), tokens 1.. are its accepted drafts.  For
+ * every layer l, KV head g and kept j, the rows k_new / v_new [l][q_offsets[r] + j][g] are
+ * copied into the cache slot of position p = kv_len[r] + j (page block_table[r][p / page_size],
+ * row p % page_size), and kv_len_out[r] = kv_len[r] + accepted_len[r] + 1.  Rejected drafts are
+ * never written, so nothing is rolled back.  (The pages describe no cache layout or interface:
+ * this reading is listed in the design notes.)
+ *
+ * k_new, v_new: `layers` blocks [T_cap][Hkv][D] of `dtype`, new_layer_stride ELEMENTS apart;
+ * kv_pages: `layers` caches [num_pages][2][Hkv][page_size][D], cache_layer_stride ELEMENTS apart
+ * (callers whose per-layer caches are separate allocations call once per layer, layers = 1);
+ * block_table int32 [R][max_pages] must already hold pages for positions up to
+ * kv_len[r] + accepted_len[r]; kv_len, q_offsets, accepted_len int32 (read); kv_len_out int32
+ * [R] (written; must not alias kv_len).  D * element size must be a multiple of 16 bytes and
+ * every tensor 16-byte aligned.
+ * Bad device data (q_offsets malformed, accepted_len outside [0, verify_len], a kept position
+ * beyond the block table, a page outside [0, num_pages)) sets DSPARK_DERR_OFFSETS / _ACCEPTED /
+ * _KV_LEN / _PAGE; that request is left untouched and kv_len_out[r] = kv_len[r].
+ */
+int dspark_kv_commit(const void *k_new, const void *v_new, int64_t new_layer_stride,
+                     void *kv_pages, int64_t num_pages, int64_t cache_layer_stride, int layers,
+                     const int32_t *block_table, int max_pages, const int32_t *kv_len,
+                     const int32_t *q_offsets, const int32_t *accepted_len, int R, int T_cap,
+                     int Hkv, int D, int K, int page_size, int dtype, int32_t *kv_len_out,
+                     dspark_stream_t stream);
 
 /*
  * dspark_read_error — synchronise `stream`, return the current device's sticky error word

@@ -10,6 +10,7 @@
 #include "attn_common.cuh"
 #include "attn_generic.cuh"
 #include "accept.cuh"
+#include "kv_commit.cuh"
 #include "attn_tc.cuh"
 
 #include <cudaTypedefs.h>
@@ -291,6 +292,41 @@ int dspark_accept(const void *target_logits, const void *draft_logits, int dtype
   };
   if (dtype == DSPARK_BF16) return run(__nv_bfloat16());
   return run(float());
+}
+
+int dspark_kv_commit(const void *k_new, const void *v_new, int64_t new_layer_stride,
+                     void *kv_pages, int64_t num_pages, int64_t cache_layer_stride, int layers,
+                     const int32_t *block_table, int max_pages, const int32_t *kv_len,
+                     const int32_t *q_offsets, const int32_t *accepted_len, int R, int T_cap,
+                     int Hkv, int D, int K, int page_size, int dtype, int32_t *kv_len_out,
+                     dspark_stream_t stream) {
+  if (!k_new || !v_new || !kv_pages || !block_table || !kv_len || !q_offsets || !accepted_len ||
+      !kv_len_out || kv_len_out == kv_len)
+    return DSPARK_EINVAL;
+  if (dtype != DSPARK_BF16 && dtype != DSPARK_F32) return DSPARK_EINVAL;
+  const int esz = dtype == DSPARK_BF16 ? 2 : 4;
+  if (R < 1 || T_cap < R || Hkv < 1 || D < 1 || K < 1 || K > DSPARK_MAX_K || page_size < 1 ||
+      max_pages < 1 || num_pages < 1 || layers < 1 || layers > 65535 || (D * esz) % 16 != 0)
+    return DSPARK_EINVAL;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(kv_pages)) return DSPARK_EINVAL;
+  const int64_t new_elems = (int64_t)T_cap * Hkv * D;
+  const int64_t cache_elems = num_pages * 2 * Hkv * page_size * (int64_t)D;
+  if (layers > 1 && (new_layer_stride < new_elems || cache_layer_stride < cache_elems ||
+                     (new_layer_stride * esz) % 16 != 0 || (cache_layer_stride * esz) % 16 != 0))
+    return DSPARK_EINVAL;
+  CommitArgs a;
+  a.k_new = static_cast<const char *>(k_new);
+  a.v_new = static_cast<const char *>(v_new);
+  a.kv = static_cast<char *>(kv_pages);
+  a.new_layer_bytes = new_layer_stride * esz;
+  a.cache_layer_bytes = cache_layer_stride * esz;
+  a.num_pages = num_pages;
+  a.block_table = block_table; a.kv_len = kv_len; a.q_offsets = q_offsets;
+  a.accepted_len = accepted_len; a.kv_len_out = kv_len_out;
+  a.max_pages = max_pages; a.R = R; a.T_cap = T_cap; a.Hkv = Hkv; a.D = D; a.K = K;
+  a.page_size = page_size; a.esz = esz;
+  kv_commit_kernel<<<dim3(R, layers), kCommitThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  return launch_status();
 }
 
 int dspark_read_error(int32_t *host_code, dspark_stream_t stream) {

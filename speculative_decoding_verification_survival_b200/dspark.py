@@ -24,7 +24,7 @@ DSPARK_ACCEPT_NOALLOC_MAX_ROWS = 65536
 DEVICE_ERROR_BITS = {
     1 << 0: "CONF", 1 << 1: "TABLE", 1 << 2: "KV_LEN", 1 << 3: "PAGE", 1 << 4: "MARKER",
     1 << 5: "OFFSETS", 1 << 6: "VERIFY_LEN", 1 << 7: "TOKEN", 1 << 8: "LOGITS",
-    1 << 9: "TIMEOUT",
+    1 << 9: "TIMEOUT", 1 << 10: "ACCEPTED",
 }
 
 
@@ -61,6 +61,8 @@ _SIGS = {
     "dspark_accept": ([_p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _f, _p, _p, _p, _p, _sz,
                        _p], _i),
     "dspark_read_error": ([ctypes.POINTER(ctypes.c_int32), _p], _i),
+    "dspark_kv_commit": ([_p, _p, _i64, _p, _i64, _i64, _i, _p, _i, _p, _p, _p, _i, _i, _i, _i,
+                          _i, _i, _i, _p, _p], _i),
     "dspark_accept_noalloc": ([_p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _f, _p, _p, _p,
                                _p], _i),
 }
@@ -199,3 +201,29 @@ def dspark_accept_noalloc(target_logits, draft_logits, draft_tokens, verify_len,
           _dtype_code(target_logits), V, R, K, T_cap, _ptr(draft_tokens), _ptr(verify_len),
           _ptr(q_offsets), _ptr(u_acc), _ptr(u_res), float(temperature), _ptr(accepted_len),
           _ptr(out_tokens), _ptr(n_out), _stream(stream))
+
+
+def dspark_kv_commit(k_new, v_new, kv_pages, block_table, kv_len, q_offsets, accepted_len, K,
+                     kv_len_out, stream=None):
+    """Kept verify rows into the paged cache.  k_new / v_new [layers][T_cap][Hkv][D] (or
+    [T_cap][Hkv][D] for one layer); kv_pages [layers][P][2][Hkv][page][D] (or one cache);
+    kv_len_out int32 [R] must not alias kv_len."""
+    if k_new.dim() == 3:
+        k_new, v_new = k_new.unsqueeze(0), v_new.unsqueeze(0)
+    if kv_pages.dim() == 5:
+        kv_pages = kv_pages.unsqueeze(0)
+    layers, T_cap, Hkv, D = k_new.shape
+    if kv_pages.shape[0] != layers or v_new.shape != k_new.shape:
+        raise ValueError("k_new, v_new and kv_pages must have the same number of layers")
+    _, num_pages, _, _, page_size, _ = kv_pages.shape
+    R, max_pages = block_table.shape
+    for t in (v_new, kv_pages):
+        if t.dtype != k_new.dtype:
+            raise TypeError("k_new, v_new and kv_pages must share a dtype")
+    for t, n in ((block_table, "block_table"), (kv_len, "kv_len"), (q_offsets, "q_offsets"),
+                 (accepted_len, "accepted_len"), (kv_len_out, "kv_len_out")):
+        _check(t, torch.int32, n)
+    _call("dspark_kv_commit", _ptr(k_new), _ptr(v_new), k_new[0].numel(), _ptr(kv_pages),
+          num_pages, kv_pages[0].numel(), layers, _ptr(block_table), max_pages, _ptr(kv_len),
+          _ptr(q_offsets), _ptr(accepted_len), R, T_cap, Hkv, D, int(K), page_size,
+          _dtype_code(k_new), _ptr(kv_len_out), _stream(stream))

@@ -56,6 +56,12 @@ class VerifyStep:
                          self.q_offsets, u_acc, u_res, temperature, self.accepted_len,
                          self.out_tokens, self.n_out, self.accept_ws, stream)
 
+    def commit(self, k_new, v_new, kv_pages, block_table, kv_len, kv_len_out, stream=None):
+        """Append each request's kept verify rows (token 0 and its accepted drafts) to its paged
+        cache for every layer; kv_len_out = kv_len + accepted + 1."""
+        _d.dspark_kv_commit(k_new, v_new, kv_pages, block_table, kv_len, self.q_offsets,
+                            self.accepted_len, self.K, kv_len_out, stream)
+
     def run(self, conf_ring, round_idx, kv_len, t_ms, layers, kv_pages_per_layer, block_table,
             attn_out, target_logits, draft_logits, draft_tokens, u_acc, u_res, temperature,
             stream=None) -> int:

@@ -97,3 +97,23 @@ def test_host_validation_rejects_before_launch(lib):
     assert h(P, P, 1, 32, 4, 5, 24, P, P, P, P, P, 1.0, P, P, P, P, 8, None) == -3
     # NaN temperature
     assert h(P, P, 1, 32, 4, 5, 24, P, P, P, P, P, float("nan"), P, P, P, P, 4096, None) == -1
+
+
+def test_kv_commit_host_validation(lib):
+    from speculative_decoding_verification_survival_b200 import dspark as d
+    f = lib.dspark_kv_commit
+    f.argtypes = d._SIGS["dspark_kv_commit"][0]
+    P, Q = ctypes.c_void_p(16), ctypes.c_void_p(32)
+    base = [P, P, 0, P, 10, 0, 1, P, 4, P, P, P, 4, 24, 2, 128, 5, 64, 1, Q, None]
+    a = list(base); a[19] = P                       # kv_len_out aliases kv_len
+    assert f(*a) == -1
+    a = list(base); a[18] = 9                       # unknown dtype
+    assert f(*a) == -1
+    a = list(base); a[15] = 4                       # D * 2 bytes not a multiple of 16
+    assert f(*a) == -1
+    a = list(base); a[6] = 2                        # two layers with no layer stride
+    assert f(*a) == -1
+    a = list(base); a[0] = ctypes.c_void_p(18)      # misaligned k_new
+    assert f(*a) == -1
+    a = list(base); a[16] = 17                      # K above the supported maximum
+    assert f(*a) == -1

@@ -93,12 +93,13 @@ def step_time_table(cfg: StepConfig, T_cap: Optional[int] = None) -> np.ndarray:
     return cfg.t_base_ms + cfg.t_slope_ms * np.maximum(0.0, T - cfg.t_knee)
 
 
-def page_table(kv_len: np.ndarray, page_size: int, rng: np.random.Generator):
-    """Random physical placement of each request's KV pages.
+def page_table(kv_len: np.ndarray, page_size: int, rng: np.random.Generator, reserve: int = 0):
+    """Random physical placement of each request's KV pages, with room for `reserve` more
+    tokens per request (the positions a verify round may append).
 
     Returns (block_table int32 [R][max_pages] padded with -1, num_pages).
     """
-    pages_per = (kv_len.astype(np.int64) + page_size - 1) // page_size
+    pages_per = (kv_len.astype(np.int64) + reserve + page_size - 1) // page_size
     num_pages = int(pages_per.sum())
     max_pages = max(1, int(pages_per.max()) if len(pages_per) else 1)
     perm = rng.permutation(num_pages).astype(np.int32)
@@ -168,7 +169,7 @@ def build_step_inputs(cfg: StepConfig, device="cpu", seed: int = 0, layers: Opti
     R, K, V = cfg.R, cfg.K, cfg.V
 
     kv_len = kv_lengths(cfg, rng)
-    table, num_pages = page_table(kv_len, cfg.page_size, rng)
+    table, num_pages = page_table(kv_len, cfg.page_size, rng, reserve=cfg.K + 1)
     history = confidences(cfg, rng, rounds)
     round_idx = rounds - 1
     ring = conf_ring(history, round_idx)
