@@ -26,3 +26,4 @@ from .schedule import (survival_ref, schedule_ref, schedule_bruteforce, flatten_
 from .attention import attn_ref_flat, attn_ref_dense  # noqa: F401
 from .accept import accept_ref  # noqa: F401
 from .kv_commit import kv_commit_ref  # noqa: F401
+from .calibration import calibrate_ref, fit_temperature_ref, outcomes_from_accept  # noqa: F401
