@@ -11,6 +11,8 @@
  *   dspark_accept          exact acceptance rule, longest accepted prefix, residual / bonus
  *                          resampling (or greedy verification)
  *   dspark_kv_commit       the kept tokens' K/V into the paged cache (after acceptance)
+ *   dspark_calibrate_confidence / dspark_fit_temperature
+ *                          temporal temperature scaling of the confidence head
  *
  * Conventions shared by every entry point:
  *   - Every pointer argument is DEVICE memory owned by the caller, unless stated otherwise.
@@ -75,7 +77,8 @@ enum dspark_device_error {
   DSPARK_DERR_TOKEN = 1 << 7,       /* a draft token outside [0, V) */
   DSPARK_DERR_LOGITS = 1 << 8,      /* a logit row whose maximum is not finite */
   DSPARK_DERR_TIMEOUT = 1 << 9,     /* a bounded in-kernel wait expired; results undefined */
-  DSPARK_DERR_ACCEPTED = 1 << 10    /* an accepted length outside [0, verify_len] */
+  DSPARK_DERR_ACCEPTED = 1 << 10    /* an accepted length outside [0, verify_len] (or a
+                                       verify length outside [0, K] in a temperature fit) */
 };
 
 #define DSPARK_CONF_LAG 2             /* rounds between producing and consuming confidences */
@@ -277,6 +280,38 @@ int dspark_kv_commit(const void *k_new, const void *v_new, int64_t new_layer_str
                      const int32_t *q_offsets, const int32_t *accepted_len, int R, int T_cap,
                      int Hkv, int D, int K, int page_size, int dtype, int32_t *kv_len_out,
                      dspark_stream_t stream);
+
+/*
+ * dspark_calibrate_confidence — temporal temperature scaling of raw confidence logits.
+ *
+ * Defined by [P1 "2. 置信度调度验证": a post-hoc calibration, "temporal temperature scaling",
+ * corrects the raw confidence head's over-confidence] with [P2 §3.2: the confidence of block
+ * position k is the acceptance probability given an accepted prefix].  Reading (the pages give
+ * only the name): conf[r][k] = sigmoid(logits[r][k] / tau[k]), one temperature per block
+ * position.  Evaluated in float64 and rounded to float32; write the result into the slot of the
+ * confidence ring that dspark_schedule reads two rounds later.
+ * logits float32 [R][K], tau float32 [K], conf float32 [R][K] (device).  A temperature that is
+ * not a positive finite number, or a NaN logit, gives 0 and sets DSPARK_DERR_CONF.
+ */
+int dspark_calibrate_confidence(const float *logits, const float *tau, int R, int K, float *conf,
+                                dspark_stream_t stream);
+
+/*
+ * dspark_fit_temperature — maximum-likelihood temperatures from observed accept outcomes.
+ *
+ * Same passages and reading as above.  Sample i (one verified request) verified verify_len[i]
+ * drafts and accepted accepted_len[i] of them; its block position k (0-based column) is
+ * observed iff k + 1 <= min(accepted_len[i] + 1, verify_len[i]), accepted iff
+ * k + 1 <= accepted_len[i].  tau[k] = 1 / beta minimises
+ * sum_observed log(1 + exp(-s * beta * logits[i][k])) (s = +1 accepted, -1 rejected) over
+ * beta in [1/64, 64]; a position without observations or with all-zero observed logits gets 1.
+ * logits float32 [N][K] (the raw logits the head produced for those requests), verify_len and
+ * accepted_len int32 [N], tau float32 [K] out (device).  Samples with lengths outside
+ * 0 <= accepted_len <= verify_len <= K are ignored and set DSPARK_DERR_ACCEPTED.
+ */
+int dspark_fit_temperature(const float *logits, const int32_t *verify_len,
+                           const int32_t *accepted_len, int N, int K, float *tau,
+                           dspark_stream_t stream);
 
 /*
  * dspark_read_error — synchronise `stream`, return the current device's sticky error word

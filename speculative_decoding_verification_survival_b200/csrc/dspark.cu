@@ -11,6 +11,7 @@
 #include "attn_generic.cuh"
 #include "accept.cuh"
 #include "kv_commit.cuh"
+#include "calibrate.cuh"
 #include "attn_tc.cuh"
 
 #include <cudaTypedefs.h>
@@ -326,6 +327,26 @@ int dspark_kv_commit(const void *k_new, const void *v_new, int64_t new_layer_str
   a.max_pages = max_pages; a.R = R; a.T_cap = T_cap; a.Hkv = Hkv; a.D = D; a.K = K;
   a.page_size = page_size; a.esz = esz;
   kv_commit_kernel<<<dim3(R, layers), kCommitThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  return launch_status();
+}
+
+int dspark_calibrate_confidence(const float *logits, const float *tau, int R, int K, float *conf,
+                                dspark_stream_t stream) {
+  if (!logits || !tau || !conf || R < 1 || K < 1 || K > DSPARK_MAX_K) return DSPARK_EINVAL;
+  const int n = R * K;
+  const int blocks = std::min((n + 255) / 256, 1024);
+  calibrate_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(logits, tau, R, K,
+                                                                                 conf);
+  return launch_status();
+}
+
+int dspark_fit_temperature(const float *logits, const int32_t *verify_len,
+                           const int32_t *accepted_len, int N, int K, float *tau,
+                           dspark_stream_t stream) {
+  if (!logits || !verify_len || !accepted_len || !tau || N < 1 || K < 1 || K > DSPARK_MAX_K)
+    return DSPARK_EINVAL;
+  fit_temperature_kernel<<<K, kFitThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      logits, verify_len, accepted_len, N, K, tau);
   return launch_status();
 }
 

@@ -61,6 +61,8 @@ _SIGS = {
     "dspark_accept": ([_p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _f, _p, _p, _p, _p, _sz,
                        _p], _i),
     "dspark_read_error": ([ctypes.POINTER(ctypes.c_int32), _p], _i),
+    "dspark_calibrate_confidence": ([_p, _p, _i, _i, _p, _p], _i),
+    "dspark_fit_temperature": ([_p, _p, _p, _i, _i, _p, _p], _i),
     "dspark_kv_commit": ([_p, _p, _i64, _p, _i64, _i64, _i, _p, _i, _p, _p, _p, _i, _i, _i, _i,
                           _i, _i, _i, _p, _p], _i),
     "dspark_accept_noalloc": ([_p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _f, _p, _p, _p,
@@ -227,3 +229,27 @@ def dspark_kv_commit(k_new, v_new, kv_pages, block_table, kv_len, q_offsets, acc
           num_pages, kv_pages[0].numel(), layers, _ptr(block_table), max_pages, _ptr(kv_len),
           _ptr(q_offsets), _ptr(accepted_len), R, T_cap, Hkv, D, int(K), page_size,
           _dtype_code(k_new), _ptr(kv_len_out), _stream(stream))
+
+
+def dspark_calibrate_confidence(logits, tau, conf, stream=None):
+    """conf[r][k] = sigmoid(logits[r][k] / tau[k]); logits / conf float32 [R][K] (conf may be a
+    slot of the confidence ring), tau float32 [K]."""
+    R, K = logits.shape
+    for t, n in ((logits, "logits"), (tau, "tau"), (conf, "conf")):
+        _check(t, torch.float32, n)
+    if tuple(conf.shape) != (R, K) or tau.numel() != K:
+        raise ValueError("logits, conf must be [R][K] and tau [K]")
+    _call("dspark_calibrate_confidence", _ptr(logits), _ptr(tau), R, K, _ptr(conf),
+          _stream(stream))
+
+
+def dspark_fit_temperature(logits, verify_len, accepted_len, tau, stream=None):
+    """Maximum-likelihood per-position temperatures from N verified requests' raw confidence
+    logits [N][K] (float32), verify_len / accepted_len int32 [N]; writes tau float32 [K]."""
+    N, K = logits.shape
+    _check(logits, torch.float32, "logits")
+    _check(tau, torch.float32, "tau")
+    _check(verify_len, torch.int32, "verify_len")
+    _check(accepted_len, torch.int32, "accepted_len")
+    _call("dspark_fit_temperature", _ptr(logits), _ptr(verify_len), _ptr(accepted_len), N, K,
+          _ptr(tau), _stream(stream))
