@@ -2,7 +2,8 @@
 
 The compute lives in libdspark.so (CUDA kernels behind the C ABI declared in include/dspark.h);
 `dspark` is its thin ctypes binding (importing it fails loudly when the library is missing) and
-`step.VerifyStep` issues one whole verify step.  `build` compiles the library in-tree.
+`step.VerifyStep` issues one whole verify step and `pipeline.RoundPipeline` replays verify rounds
+as CUDA graphs chained on the device.  `build` compiles the library in-tree.
 """
 import importlib
 
@@ -12,4 +13,6 @@ def __getattr__(name):
         return importlib.import_module(".dspark", __name__)
     if name == "VerifyStep":
         return importlib.import_module(".step", __name__).VerifyStep
+    if name == "RoundPipeline":
+        return importlib.import_module(".pipeline", __name__).RoundPipeline
     raise AttributeError(name)

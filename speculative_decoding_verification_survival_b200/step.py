@@ -62,6 +62,24 @@ class VerifyStep:
         _d.dspark_kv_commit(k_new, v_new, kv_pages, block_table, kv_len, self.q_offsets,
                             self.accepted_len, self.K, kv_len_out, stream)
 
+    def capture(self, enqueue, warmup: int = 1) -> torch.cuda.CUDAGraph:
+        """Capture `enqueue()` — any sequence of this object's calls on the current stream — as
+        one CUDA graph (after `warmup` eager runs on the capture stream).  Every launch is sized
+        by capacities (R, K, T_cap, ...), never by device results, so the graph stays valid for
+        whatever data the same buffers hold when it is replayed with `graph.replay()`."""
+        dev = self.q_offsets.device
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            for _ in range(warmup):
+                enqueue()
+        torch.cuda.current_stream(dev).wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            enqueue()
+        torch.cuda.current_stream(dev).wait_stream(s)
+        return g
+
     def run(self, conf_ring, round_idx, kv_len, t_ms, layers, kv_pages_per_layer, block_table,
             attn_out, target_logits, draft_logits, draft_tokens, u_acc, u_res, temperature,
             stream=None) -> int:

@@ -1,0 +1,97 @@
+"""Verify rounds as CUDA-graph replays (pipeline.RoundPipeline) against the same rounds run
+eagerly: bit-identical outputs round after round, with the committed cache lengths and pages
+carried on the device; plus a whole step captured with VerifyStep.capture."""
+import numpy as np
+import pytest
+import torch
+
+from tests.gpu_support import binding, host, new_step
+from workloads.configs import QWEN3_4B
+from workloads.generate import build_step_inputs, flatten_target
+
+pytestmark = pytest.mark.gpu
+
+
+def _state(cfg, seed, layers):
+    from speculative_decoding_verification_survival_b200 import RoundPipeline
+    inp = build_step_inputs(cfg, "cuda", seed=seed, layers=layers, kv_copies=1,
+                            reserve_tokens=8 * (cfg.K + 1))
+    step = new_step(cfg)
+    caches = torch.stack([inp.kv_caches[0].clone() for _ in range(layers)])
+    attn_out = torch.zeros_like(inp.q)
+    tflat = torch.empty((cfg.T_cap, cfg.V), dtype=inp.target_block.dtype, device="cuda")
+    pipe = RoundPipeline(step, inp.conf_ring.clone(), inp.t_ms, inp.kv_len.clone(),
+                         inp.block_table, inp.q.clone(), inp.k_new.clone(), inp.v_new.clone(),
+                         caches, attn_out, tflat, inp.draft_logits.clone(), inp.draft_tokens.clone(),
+                         inp.u_acc.clone(), inp.u_res.clone(), cfg.temperature)
+    return inp, pipe
+
+
+def _refill(pipe, inp, cfg, rnd):
+    """New inputs for round `rnd` (the engine's job): queries, new K/V, drafts, uniforms,
+    logits laid out for the lengths the round will schedule, a fresh confidence slot."""
+    g = torch.Generator(device="cuda").manual_seed(100 + rnd)
+    for t in (pipe.q, pipe.k_new, pipe.v_new):
+        t.copy_(torch.randn(t.shape, generator=g, device="cuda").to(t.dtype))
+    pipe.u_acc.copy_(torch.rand(pipe.u_acc.shape, generator=g, device="cuda"))
+    pipe.u_res.copy_(torch.rand(pipe.u_res.shape, generator=g, device="cuda"))
+    pipe.draft_tokens.copy_(torch.randint(0, cfg.V, pipe.draft_tokens.shape, generator=g,
+                                          device="cuda", dtype=torch.int32))
+    pipe.draft_logits.copy_(torch.randn(pipe.draft_logits.shape, generator=g, device="cuda")
+                            .to(pipe.draft_logits.dtype) * 3)
+    pipe.target_logits.copy_(torch.randn(pipe.target_logits.shape, generator=g, device="cuda")
+                             .to(pipe.target_logits.dtype) * 3)
+    pipe.conf_ring[rnd % pipe.ring_depth].copy_(
+        torch.sigmoid(torch.randn(pipe.conf_ring.shape[1:], generator=g, device="cuda") + 2))
+
+
+def test_graph_rounds_match_eager_rounds_bit_for_bit():
+    cfg = QWEN3_4B.with_(R=12, kv_dist=("uniform", 40, 700), V=256, layers=3)
+    inp_a, eager = _state(cfg, 7, 3)
+    inp_b, graph = _state(cfg, 7, 3)
+    for rnd in range(5):
+        _refill(eager, inp_a, cfg, rnd)
+        _refill(graph, inp_b, cfg, rnd)
+        eager.enqueue(rnd)
+        graph.round(rnd)
+        torch.cuda.synchronize()
+        for name in ("kv_len", "attn_out", "kv_caches"):
+            assert torch.equal(getattr(eager, name), getattr(graph, name)), (rnd, name)
+        for name in ("verify_len", "accepted_len", "out_tokens", "n_out", "markers"):
+            assert torch.equal(getattr(eager.step, name), getattr(graph.step, name)), (rnd, name)
+    # the cache lengths advanced by the kept tokens each round
+    assert torch.all(graph.kv_len > inp_b.kv_len)
+    assert binding().dspark_read_error() == 0
+
+
+def test_captured_step_replays_the_eager_step():
+    cfg = QWEN3_4B.with_(R=20, kv_dist=("uniform", 100, 900), V=512)
+    inp = build_step_inputs(cfg, "cuda", seed=3, layers=2)
+    step = new_step(cfg)
+    step.schedule(inp.conf_ring, inp.round_idx, inp.kv_len, inp.t_ms)
+    torch.cuda.synchronize()
+    tflat = flatten_target(inp.target_block, host(step.verify_len).astype(np.int64), cfg.T_cap)
+    outs = [torch.empty_like(inp.q[0]) for _ in range(2)]
+
+    def enqueue():
+        step.schedule(inp.conf_ring, inp.round_idx, inp.kv_len, inp.t_ms)
+        step.plan(inp.kv_len)
+        for layer in range(2):
+            step.attention(inp.q[layer], inp.k_new[layer], inp.v_new[layer], inp.kv_caches[0],
+                           inp.block_table, inp.kv_len, outs[layer])
+        step.accept(tflat, inp.draft_logits, inp.draft_tokens, inp.u_acc, inp.u_res,
+                    cfg.temperature)
+
+    enqueue()
+    torch.cuda.synchronize()
+    ref = [o.clone() for o in outs] + [step.accepted_len.clone(), step.out_tokens.clone()]
+    for o in outs:
+        o.zero_()
+    step.accepted_len.zero_()
+    step.out_tokens.zero_()
+    g = step.capture(enqueue)
+    g.replay()
+    torch.cuda.synchronize()
+    got = outs + [step.accepted_len, step.out_tokens]
+    for a, b in zip(ref, got):
+        assert torch.equal(a, b)

@@ -158,8 +158,10 @@ def sample_draft_tokens(draft_logits: torch.Tensor, temperature: float,
 
 
 def build_step_inputs(cfg: StepConfig, device="cpu", seed: int = 0, layers: Optional[int] = None,
-                      rounds: int = 4, kv_copies: int = 1) -> StepInputs:
-    """All inputs of verify round `rounds - 1` of workload `cfg`."""
+                      rounds: int = 4, kv_copies: int = 1,
+                      reserve_tokens: Optional[int] = None) -> StepInputs:
+    """All inputs of verify round `rounds - 1` of workload `cfg`; the block table has room for
+    `reserve_tokens` (default K + 1) appended tokens per request."""
     device = torch.device(device)
     layers = cfg.layers if layers is None else layers
     rng = np.random.default_rng(seed)
@@ -169,7 +171,8 @@ def build_step_inputs(cfg: StepConfig, device="cpu", seed: int = 0, layers: Opti
     R, K, V = cfg.R, cfg.K, cfg.V
 
     kv_len = kv_lengths(cfg, rng)
-    table, num_pages = page_table(kv_len, cfg.page_size, rng, reserve=cfg.K + 1)
+    reserve = cfg.K + 1 if reserve_tokens is None else reserve_tokens
+    table, num_pages = page_table(kv_len, cfg.page_size, rng, reserve=reserve)
     history = confidences(cfg, rng, rounds)
     round_idx = rounds - 1
     ring = conf_ring(history, round_idx)
