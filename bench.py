@@ -4,6 +4,9 @@ A step = dspark_schedule + dspark_verify_attn_plan + `layers` x dspark_verify_at
 over one batch of seeded synthetic inputs already resident in HBM.  Metric: verified draft
 tokens/s per verify step (sum of scheduled verify lengths / step time), plus accepted and
 emitted tokens/s and the achieved HBM bandwidth of the step and of its dominant kernel.
+The timed region is one replay of the K steps captured as a CUDA graph (the library sizes every
+launch by capacity, so consecutive steps need no host involvement); the eager step time is
+reported beside it.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dspark|reference]
                     [--workload qwen3-4b-64req] [--layers 36]
@@ -195,11 +198,11 @@ def run_dspark(args, rank, world, device):
         # the layer calls run back to back (each may start its prologue under the previous
         # one's tail); events bracket the whole run of them, not each call
         if ev is not None:
-            ev[0].record(stream)
+            ev[0].record()
         for (q, kn, vn), kv in zip(layers, caches):
             step.attention(q, kn, vn, kv, inp.block_table, inp.kv_len, attn_out)
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record()
         step.accept(tflat, dlog, inp.draft_tokens, inp.u_acc, inp.u_res, cfg.temperature)
 
     for _ in range(args.warmup):
@@ -209,22 +212,43 @@ def run_dspark(args, rank, world, device):
         torch.distributed.barrier()
 
     launches_per_step = 2 + cfg.layers + 2
-    ev_attn = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    # eager steps, for reference (every launch enqueued from the host)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_eager = min(args.steps, 10)
+    e0.record(stream)
+    for _ in range(n_eager):
+        one_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_eager = e0.elapsed_time(e1) / n_eager
+
+    # the timed region: the K steps captured as one CUDA graph (every launch is sized by
+    # capacities, so the steps need nothing from the host) and replayed once; events inside
+    # the graph bracket each step's run of attention calls
+    ev_attn = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
                for _ in range(args.steps)]
+
+    def timed_steps():
+        for s in range(args.steps):
+            one_step(ev_attn[s])
+
+    graph = step.capture(timed_steps, warmup=0)
+    graph.replay()          # first replay uploads the graph; untimed
+    torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clk:
         torch.cuda.synchronize()
         if world > 1:
             torch.distributed.barrier()
         t0.record(stream)
-        for s in range(args.steps):
-            one_step(ev_attn[s])
+        graph.replay()
         t1.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     ms_total = t0.elapsed_time(t1)
     attn_ms = [ev[0].elapsed_time(ev[1]) / cfg.layers for ev in ev_attn]
+    del graph
 
     # end to end through the public step API with host buffers (pinned), copies inside
     e2e = run_e2e(args, cfg, inp, step, layers, caches, tflat, dlog, L, world, device)
@@ -232,6 +256,7 @@ def run_dspark(args, rank, world, device):
     kv_len = inp.kv_len.cpu().numpy()
     acc = step.accepted_len.cpu().numpy()
     res = dict(ms_total=ms_total, attn_ms=float(np.mean(attn_ms)), L=L, kv_len=kv_len, acc=acc,
+               ms_eager=ms_eager,
                clocks=clk.summary(), launches=launches_per_step * args.steps, e2e=e2e,
                attn_bytes=attn_bytes(kv_len, L, cfg),
                step_bytes=cfg.layers * attn_bytes(kv_len, L, cfg) + logits_bytes(L, cfg, greedy),
@@ -431,6 +456,8 @@ def main():
                      h2d_bytes_per_step=res["e2e"]["h2d"], d2h_bytes_per_step=res["e2e"]["d2h"],
                      ms_per_step=e2e_ms, results_match=res["e2e"]["ok"]),
             gpu_launches=res["launches"] * world,
+            launch=dict(timed="one CUDA graph of the K steps, replayed once",
+                        ms_per_step_eager=res["ms_eager"]),
             clocks=res["clocks"])
         if not args.no_cpu_baseline:
             v, desc, cores, step_s = cpu_baseline(cfg)
