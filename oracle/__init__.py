@@ -27,3 +27,4 @@ from .attention import attn_ref_flat, attn_ref_dense  # noqa: F401
 from .accept import accept_ref  # noqa: F401
 from .kv_commit import kv_commit_ref  # noqa: F401
 from .calibration import calibrate_ref, fit_temperature_ref, outcomes_from_accept  # noqa: F401
+from .draft import markov_draft_ref  # noqa: F401
