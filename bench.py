@@ -252,11 +252,12 @@ def run_dspark(args, rank, world, device):
 
     # end to end through the public step API with host buffers (pinned), copies inside
     e2e = run_e2e(args, cfg, inp, step, layers, caches, tflat, dlog, L, world, device)
+    draft_ms = time_markov_draft(cfg, device) if cfg.dtype == "bf16" and cfg.V % 8 == 0 else None
 
     kv_len = inp.kv_len.cpu().numpy()
     acc = step.accepted_len.cpu().numpy()
     res = dict(ms_total=ms_total, attn_ms=float(np.mean(attn_ms)), L=L, kv_len=kv_len, acc=acc,
-               ms_eager=ms_eager,
+               ms_eager=ms_eager, draft_ms=draft_ms,
                clocks=clk.summary(), launches=launches_per_step * args.steps, e2e=e2e,
                attn_bytes=attn_bytes(kv_len, L, cfg),
                step_bytes=cfg.layers * attn_bytes(kv_len, L, cfg) + logits_bytes(L, cfg, greedy),
@@ -362,6 +363,34 @@ def cpu_baseline(cfg, max_seconds: float = 20.0):
     return float(L.sum()) / step_s, desc, 1, step_s
 
 
+def time_markov_draft(cfg, device, rounds: int = 10, rank: int = 64) -> float:
+    """ms per round of the synthetic Markov-head draft step (the drafter's sequential part:
+    K positions of block logits + a rank-64 previous-token transition, bf16 rounding and
+    Gumbel-max sampling) for the workload's R, K, V; weights are random multiples of 1/16."""
+    from speculative_decoding_verification_survival_b200 import dspark as d
+    g = torch.Generator(device=device).manual_seed(0)
+    R, K, V = cfg.R, cfg.K, cfg.V
+    B = (torch.randn((R, K, V), generator=g, device=device) * 3).to(torch.bfloat16)
+    E = (torch.randint(-16, 17, (V, rank), generator=g, device=device).float() / 16).to(torch.bfloat16)
+    U = (torch.randint(-16, 17, (rank, V), generator=g, device=device).float() / 16).to(torch.bfloat16)
+    x0 = torch.randint(0, V, (R,), generator=g, device=device, dtype=torch.int32)
+    out = torch.empty_like(B)
+    tok = torch.empty((R, K), dtype=torch.int32, device=device)
+    ws = torch.empty(d.dspark_markov_draft_workspace_bytes(R, V), dtype=torch.uint8, device=device)
+    tau = cfg.temperature
+    for i in range(3):
+        d.dspark_markov_draft(B, E, U, x0, tau, i, 0, out, tok, ws)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(rounds):
+        d.dspark_markov_draft(B, E, U, x0, tau, i, 0, out, tok, ws)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / rounds
+    del B, E, U, out
+    return ms
+
+
 def reduce_replicas(ms_step, attn_ms, e2e_ms, L_sum, acc_sum, R, world, device):
     """Combine independent replicas: times are the max over ranks (the job waits for the
     slowest), token and request counts are summed (every rank verifies its own batch)."""
@@ -458,6 +487,10 @@ def main():
             gpu_launches=res["launches"] * world,
             launch=dict(timed="one CUDA graph of the K steps, replayed once",
                         ms_per_step_eager=res["ms_eager"]),
+            draft_step=None if res["draft_ms"] is None else dict(
+                ms_per_round=res["draft_ms"], share_of_verify_step=res["draft_ms"] / ms_step,
+                model="Markov head: block logits (given) + rank-64 previous-token transition, "
+                      "bf16 rounding, Gumbel-max; not part of the timed step"),
             clocks=res["clocks"])
         if not args.no_cpu_baseline:
             v, desc, cores, step_s = cpu_baseline(cfg)

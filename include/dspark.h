@@ -13,6 +13,7 @@
  *   dspark_kv_commit       the kept tokens' K/V into the paged cache (after acceptance)
  *   dspark_calibrate_confidence / dspark_fit_temperature
  *                          temporal temperature scaling of the confidence head
+ *   dspark_markov_draft    synthetic Markov-head draft step (cost of the drafter's sequential part)
  *
  * Conventions shared by every entry point:
  *   - Every pointer argument is DEVICE memory owned by the caller, unless stated otherwise.
@@ -312,6 +313,33 @@ int dspark_calibrate_confidence(const float *logits, const float *tau, int R, in
 int dspark_fit_temperature(const float *logits, const int32_t *verify_len,
                            const int32_t *accepted_len, int N, int K, float *tau,
                            dspark_stream_t stream);
+
+/*
+ * dspark_markov_draft — synthetic Markov-head draft step (the drafter's sequential part).
+ *
+ * Defined by [P1 "1. 半自回归生成": a parallel backbone drafts the whole block and a light
+ * sequential module injects the prefix token by token; one form is a Markov head that depends
+ * only on the previous token].  Reading (no formulas or trained weights are published): block
+ * position k = 1..K of request r has draft logits z_k = bf16(B[r][k-1] + E[x_{k-1}] . U) — the
+ * backbone's block logits plus a rank-d transition term of the previous token — and
+ * x_k = argmax_v z_k[v] / temperature + g_v, g = -log(-log(u)), u from Philox4x32-10 with
+ * counter (round_idx, r, v / 4, 3 + 256 (k - 1)), key (seed, 0), word v % 4,
+ * u = ((word >> 8) + 1/2) 2^-24; temperature <= 0 takes the lowest index of the maximum of z_k.
+ * x_0 = x0[r], the request's last emitted token.  Its purpose is the cost of this sequential
+ * part next to a verify step (the backbone's block logits are an input).
+ * block_logits bf16 [R][K][V]; E bf16 [V][d]; U bf16 [d][V]; d a multiple of 8 up to 64;
+ * V a multiple of 8; block_logits, E, U and draft_logits 16-byte aligned; x0 int32 [R]; outputs
+ * draft_logits bf16
+ * [R][K][V] (the q distributions the verifier reads) and draft_tokens int32 [R][K]; ws from
+ * dspark_markov_draft_workspace_bytes(R, V).  2K + 1 launches.  An x0 outside [0, V) sets
+ * DSPARK_DERR_TOKEN and is read as token 0.
+ */
+size_t dspark_markov_draft_workspace_bytes(int R, int V);
+int dspark_markov_draft(const void *block_logits, const void *E, const void *U, int d,
+                        const int32_t *x0, int R, int K, int V, float temperature,
+                        uint32_t round_idx, uint32_t seed, void *draft_logits,
+                        int32_t *draft_tokens, void *ws, size_t ws_bytes,
+                        dspark_stream_t stream);
 
 /*
  * dspark_read_error — synchronise `stream`, return the current device's sticky error word

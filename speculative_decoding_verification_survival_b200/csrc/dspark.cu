@@ -12,6 +12,7 @@
 #include "accept.cuh"
 #include "kv_commit.cuh"
 #include "calibrate.cuh"
+#include "draft.cuh"
 #include "attn_tc.cuh"
 
 #include <cudaTypedefs.h>
@@ -347,6 +348,44 @@ int dspark_fit_temperature(const float *logits, const int32_t *verify_len,
     return DSPARK_EINVAL;
   fit_temperature_kernel<<<K, kFitThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       logits, verify_len, accepted_len, N, K, tau);
+  return launch_status();
+}
+
+size_t dspark_markov_draft_workspace_bytes(int R, int V) {
+  if (R < 1 || V < 4) return 0;
+  return draft_ws_layout(R, V, nullptr, nullptr);
+}
+
+int dspark_markov_draft(const void *block_logits, const void *E, const void *U, int d,
+                        const int32_t *x0, int R, int K, int V, float temperature,
+                        uint32_t round_idx, uint32_t seed, void *draft_logits,
+                        int32_t *draft_tokens, void *ws, size_t ws_bytes,
+                        dspark_stream_t stream) {
+  if (!block_logits || !E || !U || !x0 || !draft_logits || !draft_tokens) return DSPARK_EINVAL;
+  if (R < 1 || K < 1 || K > DSPARK_MAX_K || V < 8 || V % 8 != 0 || d < 8 || d % 8 != 0 ||
+      d > kDraftMaxRank || std::isnan(temperature) || std::isinf(temperature))
+    return DSPARK_EINVAL;
+  if (!aligned16(block_logits) || !aligned16(E) || !aligned16(U) || !aligned16(draft_logits))
+    return DSPARK_EINVAL;
+  if (!ws || !aligned16(ws) || ws_bytes < draft_ws_layout(R, V, nullptr, nullptr))
+    return DSPARK_EWORKSPACE;
+  DraftWs w;
+  draft_ws_layout(R, V, &w, ws);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int nslices = (V + kDraftSlice - 1) / kDraftSlice;
+  const bool sampled = temperature > 0.f;
+  const float inv_tau = sampled ? 1.f / temperature : 1.f;
+  const auto *b = static_cast<const __nv_bfloat16 *>(block_logits);
+  const auto *e = static_cast<const __nv_bfloat16 *>(E);
+  const auto *u = static_cast<const __nv_bfloat16 *>(U);
+  auto *o = static_cast<__nv_bfloat16 *>(draft_logits);
+  markov_init_kernel<<<(R + 255) / 256, 256, 0, s>>>(x0, R, V, w);
+  for (int k = 1; k <= K; ++k) {
+    markov_logits_kernel<<<nslices, kDraftThreads, 0, s>>>(b, e, u, d, w.xprev, R, K, V, k,
+                                                           inv_tau, sampled ? 1 : 0, round_idx,
+                                                           seed, o, w);
+    markov_select_kernel<<<R, 128, 0, s>>>(nslices, R, K, k, w, draft_tokens);
+  }
   return launch_status();
 }
 

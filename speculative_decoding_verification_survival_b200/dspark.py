@@ -61,6 +61,9 @@ _SIGS = {
     "dspark_accept": ([_p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _f, _p, _p, _p, _p, _sz,
                        _p], _i),
     "dspark_read_error": ([ctypes.POINTER(ctypes.c_int32), _p], _i),
+    "dspark_markov_draft_workspace_bytes": ([_i, _i], _sz),
+    "dspark_markov_draft": ([_p, _p, _p, _i, _p, _i, _i, _i, _f, ctypes.c_uint32, ctypes.c_uint32,
+                             _p, _p, _p, _sz, _p], _i),
     "dspark_calibrate_confidence": ([_p, _p, _i, _i, _p, _p], _i),
     "dspark_fit_temperature": ([_p, _p, _p, _i, _i, _p, _p], _i),
     "dspark_kv_commit": ([_p, _p, _i64, _p, _i64, _i64, _i, _p, _i, _p, _p, _p, _i, _i, _i, _i,
@@ -253,3 +256,24 @@ def dspark_fit_temperature(logits, verify_len, accepted_len, tau, stream=None):
     _check(accepted_len, torch.int32, "accepted_len")
     _call("dspark_fit_temperature", _ptr(logits), _ptr(verify_len), _ptr(accepted_len), N, K,
           _ptr(tau), _stream(stream))
+
+
+def dspark_markov_draft_workspace_bytes(R, V) -> int:
+    return int(_lib.dspark_markov_draft_workspace_bytes(R, V))
+
+
+def dspark_markov_draft(block_logits, E, U, x0, temperature, round_idx, seed, draft_logits,
+                        draft_tokens, ws, stream=None):
+    """Synthetic Markov-head draft: block_logits bf16 [R][K][V], E bf16 [V][d], U bf16 [d][V],
+    x0 int32 [R]; writes draft_logits bf16 [R][K][V] and draft_tokens int32 [R][K]."""
+    R, K, V = block_logits.shape
+    d = E.shape[1]
+    for t, n in ((block_logits, "block_logits"), (E, "E"), (U, "U"), (draft_logits, "draft_logits")):
+        _check(t, torch.bfloat16, n)
+    _check(x0, torch.int32, "x0")
+    _check(draft_tokens, torch.int32, "draft_tokens")
+    if tuple(U.shape) != (d, V) or E.shape[0] != V or tuple(draft_logits.shape) != (R, K, V):
+        raise ValueError("shapes: block_logits [R][K][V], E [V][d], U [d][V], draft_logits [R][K][V]")
+    _call("dspark_markov_draft", _ptr(block_logits), _ptr(E), _ptr(U), d, _ptr(x0), R, K, V,
+          float(temperature), int(round_idx) & 0xFFFFFFFF, int(seed) & 0xFFFFFFFF,
+          _ptr(draft_logits), _ptr(draft_tokens), _ptr(ws), ws.numel(), _stream(stream))
