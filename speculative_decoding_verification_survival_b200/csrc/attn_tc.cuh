@@ -11,22 +11,24 @@
 // minimises instructions per key: two 64-key pages form one 128-key tile, S = Q.K^T of a tile is
 // 8 MMAs (M 128, N 128, K 16) and O += P.V is 8 MMAs (M 128, N 128, K 16).
 //
-// Per CTA (192 threads):
-//   warp 4      TMA producer: one 64-row x 128-B box per d-half of a page's K and V tiles
-//               (128-byte swizzle) into four rings (K d-half 0/1, V d-half 0/1) of 6 page slots;
-//               the two pages of a tile go to slots 2p and 2p+1, which are contiguous in every
-//               ring, so one descriptor spans the tile.  An odd page or the verify-token unit
-//               leaves slot 2p+1 empty.  Verify tokens come through 3-D tensor maps over
-//               k_new / v_new (16 tokens of one KV head).
-//   warp 5      MMA issuer (one thread): A operands (Q, P; bf16) in tensor memory, B operands
-//               (K, V) in shared memory, fp32 accumulators in tensor memory.
-//   warps 0-3   softmax + epilogue.  TMEM lane quadrant w is readable only by warp w, so each
-//               query row is replicated C times (C = 4 for <= 32 rows, else 2): copy c lives in
-//               lanes [c*128/C, (c+1)*128/C) and handles keys [c*128/C, (c+1)*128/C) of every
-//               tile, spreading the exp2 work of a row over C SM sub-partitions.  Partial row
-//               maxima are exchanged through shared memory (named barrier); each copy writes P
-//               for its own keys (zeros elsewhere) into its own lanes, so every copy accumulates
-//               a partial O over its keys and the epilogue sums the copies.  O is rescaled in
+// Per CTA (352 threads, 11 warps):
+//   warp 8      TMA producer of K: per 64-key page, one 64-row x 128-B box per d-half (128-byte
+//               swizzle) into two rings of 6 page slots; the two pages of a tile go to slots 2p
+//               and 2p+1, which are contiguous, so one descriptor spans the tile.  An odd page
+//               or the verify-token unit leaves slot 2p+1 empty.  Verify tokens come through
+//               3-D tensor maps over k_new / v_new (16 tokens of one KV head).
+//   warp 10     TMA producer of V (same layout, its own barriers: K is released after S, V only
+//               after P.V).
+//   warp 9      MMA issuer (one thread, polling): A operands (Q, P; bf16) in tensor memory, B
+//               operands (K, V) in shared memory, fp32 accumulators in tensor memory.
+//   warps 0-7   softmax + epilogue.  TMEM lane quadrant q is readable only by warps q and q + 4,
+//               so each query row is replicated C times (C = 4 for <= 32 rows, else 2): copy c
+//               lives in lanes [c*128/C, (c+1)*128/C) and handles keys [c*128/C, (c+1)*128/C) of
+//               every tile, and the quadrant's two warps split those keys in halves, spreading
+//               the exp2 work of a row over 2C warps.  Partial row maxima are exchanged through
+//               shared memory (named barrier); each thread writes P for its keys (zeros for the
+//               other copies' keys) into its lane's P columns, so every copy accumulates a
+//               partial O over its keys and the epilogue sums the copies.  O is rescaled in
 //               TMEM only when the running maximum grows by more than 2^8.  The verify-token
 //               unit applies the causal rule from the markers (token j sees verify tokens 0..j).
 // TMEM columns: S [0,256) (two 128-column tiles), Q [256,320), P [320,384), O [384,512).
@@ -51,8 +53,10 @@ constexpr int kPairsK = kSlotsK / 2, kPairsV = kSlotsV / 2;
 constexpr int kMaxSlots = 8;
 static_assert(kSlotsK % 2 == 0 && kSlotsV % 2 == 0 && kSlotsK <= kMaxSlots && kSlotsV <= kMaxSlots,
               "slot counts");
-constexpr int kThreads = 224;
-constexpr int kSoftmaxThreads = 128;
+constexpr int kSoftmaxWarps = 8;                     // two per TMEM lane quadrant
+constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+constexpr int kWarpK = kSoftmaxWarps, kWarpMma = kSoftmaxWarps + 1, kWarpV = kSoftmaxWarps + 2;
+constexpr int kThreads = kSoftmaxThreads + 96;
 constexpr int kD = 128;
 constexpr int kNewRows = 16;                         // verify tokens per unit (K + 1 <= 16)
 constexpr uint32_t kSlotBytes = 64 * 128;            // 64 rows x 128 B: one d-half of a page
@@ -61,7 +65,7 @@ constexpr uint32_t kRingBytesV = kSlotsV * kSlotBytes;  // one V ring
 constexpr uint32_t kHalfPageBytes = 2 * kSlotBytes;  // K (or V) of a page, both d-halves
 constexpr uint32_t kNewHalfBytes = 2 * kNewRows * 128;  // K (or V) of the verify-token unit
 constexpr uint32_t kOffAux = 2 * kRingBytesK + 2 * kRingBytesV;
-constexpr uint32_t kAuxBytes = 2048;
+constexpr uint32_t kAuxBytes = 4096;
 // staging: the next piece's query rows (<= 64 x 256 B), then the epilogue's 128 x 32 fp32
 constexpr uint32_t kOffStage = kOffAux + kAuxBytes;
 constexpr uint32_t kStageBytes = 16384;
@@ -73,7 +77,7 @@ constexpr uint32_t kBarKFull = 0, kBarVFull = 64, kBarKEmpty = 128, kBarVEmpty =
                    kBarSFull = 256, kBarPFull = 272, kBarODone = 280, kBarQFull = 288,
                    kBarQEmpty = 296, kBarOFree = 304;
 constexpr uint32_t kAuxTmem = 320, kAuxAbort = 324, kAuxLast = 328, kAuxPmax = 512,
-                   kAuxLsum = 512 + 2 * 128 * 4;
+                   kAuxLsum = 512 + 2 * kSoftmaxThreads * 4;
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;
@@ -206,21 +210,24 @@ struct SoftmaxState {
   float l_part;  // partial row sum over this copy's keys
 };
 
-// One tile for the thread's lane: S slice from TMEM, masking (valid keys, causal bound), row
-// maximum across copies (named barrier 1), conditional rescale of this lane's O, P (bf16) for
-// this copy's keys into this lane's P columns.  NKC = keys per copy.  `gt` = global tile index.
+// One tile for the thread's lane and key half: S slice from TMEM, masking (valid keys, causal
+// bound), row maximum across copies and halves (named barrier 1), conditional rescale of this
+// thread's half of the lane's O, P (bf16) for its keys into the lane's P columns.  NKC = keys per
+// copy (each of the quadrant's two warps takes NKC / 2 of them).  `gt` = global tile index.
 template <int NKC>
 __device__ __forceinline__ void softmax_tile(const AttnArgs &a, SoftmaxState &st, uint32_t tmem,
                                              uint32_t lane_base, uint32_t aux, float *pmax_buf,
                                              volatile int *abort_flag, uint32_t gt, int vk,
-                                             int jrow, int t, int copy, int rho, int rpc,
+                                             int jrow, int t, int hf, int copy, int rho, int rpc,
                                              bool active) {
   constexpr int C = kTK / NKC;
+  constexpr int NKH = NKC / 2;
   const uint32_t b = gt & 1;
-  float s[NKC];
-  const uint32_t s_taddr = tmem + lane_base + kColS + b * kTK + copy * NKC;
+  float s[NKH];
+  const int key0 = copy * NKC + hf * NKH;
+  const uint32_t s_taddr = tmem + lane_base + kColS + b * kTK + key0;
 #pragma unroll
-  for (int c16 = 0; c16 < NKC / 16; ++c16) {
+  for (int c16 = 0; c16 < NKH / 16; ++c16) {
     float v[16];
     ptx::tmem_ld16(s_taddr + c16 * 16, v);
 #pragma unroll
@@ -229,17 +236,20 @@ __device__ __forceinline__ void softmax_tile(const AttnArgs &a, SoftmaxState &st
   ptx::tmem_wait_ld();
   float mx = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < NKC; ++i) {
-    const int key = copy * NKC + i;
+  for (int i = 0; i < NKH; ++i) {
+    const int key = key0 + i;
     const float x = (active && key < vk && key <= jrow) ? s[i] * a.scale_log2 : -INFINITY;
     s[i] = x;
     mx = fmaxf(mx, x);
   }
-  pmax_buf[b * 128 + t] = mx;
+  pmax_buf[b * kSoftmaxThreads + hf * 128 + t] = mx;
   ptx::named_bar_sync(1, kSoftmaxThreads);
   float mt = -INFINITY;
 #pragma unroll
-  for (int cc = 0; cc < C; ++cc) mt = fmaxf(mt, pmax_buf[b * 128 + rho + cc * rpc]);
+  for (int cc = 0; cc < C; ++cc) {
+    mt = fmaxf(mt, pmax_buf[b * kSoftmaxThreads + rho + cc * rpc]);
+    mt = fmaxf(mt, pmax_buf[b * kSoftmaxThreads + 128 + rho + cc * rpc]);
+  }
   const float m_new = fmaxf(st.m_run, mt);
   float alpha = 1.f;
   bool resc = false;
@@ -253,9 +263,9 @@ __device__ __forceinline__ void softmax_tile(const AttnArgs &a, SoftmaxState &st
   }
   // compute P before waiting for the tensor core
   float lsum = 0.f;
-  uint32_t w[NKC / 2];
+  uint32_t w[NKH / 2];
 #pragma unroll
-  for (int h = 0; h < NKC / 2; ++h) {
+  for (int h = 0; h < NKH / 2; ++h) {
     const float p0 = active ? ex2(s[2 * h] - st.m_run) : 0.f;
     const float p1 = active ? ex2(s[2 * h + 1] - st.m_run) : 0.f;
     const __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
@@ -271,9 +281,10 @@ __device__ __forceinline__ void softmax_tile(const AttnArgs &a, SoftmaxState &st
   }
   if (__any_sync(0xffffffffu, resc)) {
     // this lane's O holds the earlier tiles relative to the old maximum: rescale it in TMEM
-    const uint32_t o_taddr = tmem + lane_base + kColO;
+    // (each of the quadrant's two warps takes half of the columns)
+    const uint32_t o_taddr = tmem + lane_base + kColO + hf * 64;
 #pragma unroll 1
-    for (int c32 = 0; c32 < 4; ++c32) {
+    for (int c32 = 0; c32 < 2; ++c32) {
       float v[32];
       ptx::tmem_ld32(o_taddr + c32 * 32, v);
       ptx::tmem_wait_ld();
@@ -283,7 +294,7 @@ __device__ __forceinline__ void softmax_tile(const AttnArgs &a, SoftmaxState &st
       ptx::tmem_st<32>(o_taddr + c32 * 32, ow);
     }
   }
-  ptx::tmem_st<NKC / 2>(tmem + lane_base + kColP + copy * (NKC / 2), w);
+  ptx::tmem_st<NKH / 2>(tmem + lane_base + kColP + key0 / 2, w);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -329,12 +340,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
     *s_last = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kWarpK && lane == 0) {
     ptx::prefetch_tmap(&tmap_kv);
     ptx::prefetch_tmap(&tmap_kn);
     ptx::prefetch_tmap(&tmap_vn);
   }
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     ptx::tmem_alloc(aux + kAuxTmem, kTmemCols);
     ptx::tmem_relinquish();
     ptx::tc_fence_before();
@@ -352,13 +363,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
   it.init(a);
   int r, g, ta, tb, tiles, s0;
 
-  if (warp == 4 || warp == 6) {
+  if (warp == kWarpK || warp == kWarpV) {
     // ------------------------------------------------------------------ TMA producers
-    // warp 4 loads K, warp 6 loads V (a bulk L2 prefetch of later pages was tried and only
+    // one warp loads K, another V (a bulk L2 prefetch of later pages was tried and only
     // lengthened the loads' latency).  Tile gt
     // uses page slots 2(gt mod 3) and 2(gt mod 3) + 1 of both rings' families.
     if (lane == 0) {
-      const bool is_k = (warp == 4);
+      const bool is_k = (warp == kWarpK);
       const uint32_t full0 = is_k ? kBarKFull : kBarVFull, empty0 = is_k ? kBarKEmpty : kBarVEmpty;
       const int rg0 = is_k ? 0 : 2;
       const CUtensorMap *nmap = is_k ? &tmap_kn : &tmap_vn;
@@ -406,7 +417,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
         if (last_use[k] >= 0)
           ptx::mbar_wait(bar(full0, k), ((uint32_t)last_use[k] / nslots) & 1, &no_abort);
     }
-  } else if (warp == 5) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     // Two cursors: S(js) for the next tile whose K has landed, P.V(jp) for the oldest tile whose
     // P is written.  Whichever is ready is issued (P.V first), so a late K load never holds back
@@ -490,8 +501,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    const int t = tid;  // TMEM lane of this thread (0..127)
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int t = tid & 127;   // TMEM lane of this thread (its warp's lane quadrant)
+    const int hf = tid >> 7;   // which half of each copy's keys (and of O's columns) it takes
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(a.q);
     __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.out);
     const int G = a.G;
@@ -501,7 +513,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
     // area with asynchronous 16-byte copies, chunk c of row rq at chunk slot c ^ (rq & 7) so the
     // lane-per-row reads of q_commit spread over the banks.
     auto q_prefetch = [&](const Meta &mq, int gq) {
-      for (int idx = t; idx < mq.rows * 16; idx += kSoftmaxThreads) {
+      for (int idx = tid; idx < mq.rows * 16; idx += kSoftmaxThreads) {
         const int rq = idx >> 4, c = idx & 15;
         const int j = rq / G, i = rq % G;
         ptx::cp_async16(stage + rq * 256 + ((c ^ (rq & 7)) << 4),
@@ -517,8 +529,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       const int rq = t % (128 / mq.C);
       ptx::mbar_wait(bar(kBarQEmpty, 0), (qidx & 1) ^ 1, abort_flag);
       ptx::tc_fence_after();
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      {  // this thread writes the lane's Q columns of d-half hf
+        const int h = hf;
         uint32_t w[32];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -538,7 +550,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
     bool have = it.next(a, r, g, ta, tb, tiles, s0);
     Meta m;
     if (have) {
-      m = piece_meta(a, r, ta, tb, tiles, t == 0);
+      m = piece_meta(a, r, ta, tb, tiles, tid == 0);
       if (m.ntiles > 0) {
         q_prefetch(m, g);
         q_commit(m);
@@ -551,7 +563,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       const bool have2 = it.next(a, r2, g2, ta2, tb2, tiles2, s02);
       Meta m2;
       if (have2) {
-        m2 = piece_meta(a, r2, ta2, tb2, tiles2, t == 0);
+        m2 = piece_meta(a, r2, ta2, tb2, tiles2, tid == 0);
         if (m2.ntiles > 0) q_prefetch(m2, g2);
       }
 
@@ -572,26 +584,39 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
         ptx::tc_fence_after();
         if (j == 0) {
           // this lane's P columns outside its copy's keys must read as zero (the previous
-          // piece's P.V MMAs have completed: its epilogue waited for them)
-          uint32_t z[32];
+          // piece's P.V MMAs have completed: its epilogue waited for them).  Each of the
+          // quadrant's two warps zeroes its own key half of the other copies, so the two never
+          // write the same columns.
+          uint32_t z[16];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) z[c] = 0u;
-          ptx::tmem_st<32>(tmem + lane_base + kColP, z);
-          ptx::tmem_st<32>(tmem + lane_base + kColP + 32, z);
+          for (int c = 0; c < 16; ++c) z[c] = 0u;
+          const int ph = kTK / m.C / 4;  // P columns of one copy's key half (8 or 16)
+          for (int cc = 0; cc < m.C; ++cc) {
+            if (cc == copy) continue;
+            const uint32_t col = tmem + lane_base + kColP + cc * 2 * ph + hf * ph;
+            if (ph == 8) {
+              uint32_t z8[8];
+#pragma unroll
+              for (int c = 0; c < 8; ++c) z8[c] = 0u;
+              ptx::tmem_st<8>(col, z8);
+            } else {
+              ptx::tmem_st<16>(col, z);
+            }
+          }
         }
         if (m.C == 4)
           softmax_tile<32>(a, sm, tmem, lane_base, aux, pmax_buf, abort_flag, gt_, vk, jrow, t,
-                           copy, rho, rpc, active);
+                           hf, copy, rho, rpc, active);
         else
           softmax_tile<64>(a, sm, tmem, lane_base, aux, pmax_buf, abort_flag, gt_, vk, jrow, t,
-                           copy, rho, rpc, active);
+                           hf, copy, rho, rpc, active);
         // V rows the P.V MMA reads past the valid keys may hold anything: zero them so that
         // P = 0 times V stays 0 (the MMA reads whole 16-key steps of valid pages)
         const int vrows = cache_tile ? min(kTK, (vk + kPage - 1) / kPage * kPage) : kNewRows;
         if (vk < vrows) {
           const uint32_t pair = gt_ % kPairsV;
           ptx::mbar_wait(bar(kBarVFull, 2 * pair + vk / kPage), (gt_ / kPairsV) & 1, abort_flag);
-          for (int idx = t; idx < (vrows - vk) * 16; idx += kSoftmaxThreads) {
+          for (int idx = tid; idx < (vrows - vk) * 16; idx += kSoftmaxThreads) {
             const uint32_t row = vk + idx / 16, half = (idx % 16) / 8, c = idx % 8;
             st_shared_v4(ring(2 + half, 2 * pair) + row * 128 + c * 16, 0u, 0u, 0u, 0u);
           }
@@ -606,11 +631,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       if (have2 && m2.ntiles > 0) q_commit(m2);
 
       // ---------------------------------------------------------------- epilogue
-      // Each copy holds a partial O over its own keys.  Four rounds of 32 columns: every lane
-      // puts its columns into the staging area, then lane (copy, rho) sums the copies of row rho
-      // for its 32 / C columns of the round and writes them (bf16 output, or the fp32 partial of
-      // a split segment).
-      lsum_buf[t] = sm.l_part;
+      // Each copy holds a partial O over its own keys.  Four rounds of 32 columns: the lane's two
+      // threads put its columns into the staging area (16 each), then thread (copy, half, rho)
+      // sums the copies of row rho for its 32 / (2 C) columns of the round and writes them
+      // (bf16 output, or the fp32 partial of a split segment).
+      lsum_buf[tid] = sm.l_part;
       if (m.ntiles > 0) {
         ptx::mbar_wait(bar(kBarODone, 0), (gt + m.ntiles - 1) & 1, abort_flag);
         ptx::tc_fence_after();
@@ -621,24 +646,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       float *part = a.ws.partials + (size_t)partial_slot(blockIdx.x, s0, W) * a.rows_max * kPS;
       if (m.ntiles > 0) {
         float l = 0.f;
-        for (int cc = 0; cc < m.C; ++cc) l += lsum_buf[rho + cc * rpc];
+        for (int cc = 0; cc < m.C; ++cc) l += lsum_buf[rho + cc * rpc] + lsum_buf[128 + rho + cc * rpc];
         const float inv = 1.f / l;
         const int j = rho / G, i = rho % G;
         const size_t orow = ((size_t)(m.t0 + j) * a.Hq + g * G + i) * kD;
-        const uint32_t o_taddr = tmem + lane_base + kColO;
-        const int nc = 32 / m.C;  // columns of a round this lane finishes (8 or 16)
+        const uint32_t o_taddr = tmem + lane_base + kColO + hf * 16;
+        const int nc = 16 / m.C;  // columns of a round this thread finishes (4 or 8)
 #pragma unroll 1
         for (int c32 = 0; c32 < 4; ++c32) {
-          float o[32];
-          ptx::tmem_ld32(o_taddr + c32 * 32, o);
+          float o[16];
+          ptx::tmem_ld16(o_taddr + c32 * 32, o);
           ptx::tmem_wait_ld();
           if (c32 == 3) {  // O fully read: the next piece's P.V may overwrite it
             ptx::tc_fence_before();
             ptx::mbar_arrive(bar(kBarOFree, 0));
           }
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            st_shared_v4(stage + t * 128 + ((k ^ (t & 7)) << 4), __float_as_uint(o[4 * k]),
+          for (int k = 0; k < 4; ++k)
+            st_shared_v4(stage + t * 128 + (((hf * 4 + k) ^ (t & 7)) << 4), __float_as_uint(o[4 * k]),
                          __float_as_uint(o[4 * k + 1]), __float_as_uint(o[4 * k + 2]),
                          __float_as_uint(o[4 * k + 3]));
           ptx::named_bar_sync(2, kSoftmaxThreads);
@@ -646,7 +671,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
             float acc[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-            const int k0 = copy * (nc / 4);   // first float4 chunk of this lane's columns
+            const int k0 = (copy * 2 + hf) * (nc / 4);  // first float4 chunk of these columns
             for (int cc = 0; cc < m.C; ++cc) {
               const int row = rho + cc * rpc;
 #pragma unroll
@@ -660,7 +685,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
                 }
               }
             }
-            const int col0 = c32 * 32 + copy * nc;
+            const int col0 = c32 * 32 + (copy * 2 + hf) * nc;
             if (whole) {
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
@@ -681,21 +706,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
           }
           ptx::named_bar_sync(2, kSoftmaxThreads);  // before the next round reuses the staging
         }
-        if (active && copy == 0 && !whole) {
+        if (active && copy == 0 && hf == 0 && !whole) {
           part[(size_t)rho * kPS + kD] = sm.m_run;
           part[(size_t)rho * kPS + kD + 1] = l;
         }
         gt += m.ntiles;
       } else if (!whole) {
         // a piece holding only tail units of its segment: a partial without keys
-        for (int idx = t; idx < m.rows * kPS; idx += kSoftmaxThreads)
+        for (int idx = tid; idx < m.rows * kPS; idx += kSoftmaxThreads)
           part[idx] = (idx % kPS == kD) ? -INFINITY : 0.f;
       }
 
       if (!whole) {  // split segment: publish the partial, the last piece merges
         __threadfence();
         ptx::named_bar_sync(2, kSoftmaxThreads);
-        if (t == 0) {
+        if (tid == 0) {
           const int pieces = (s0 + tiles - 1) / W - s0 / W + 1;
           const int prev = atomicAdd(a.ws.counters + r * a.Hkv + g, 1);
           *s_last = (prev == pieces - 1);
@@ -706,17 +731,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
           const int c_first = s0 / W, c_last = (s0 + tiles - 1) / W;
           const size_t pstride = (size_t)a.rows_max * kPS;
           const float *P0 = a.ws.partials;
-          // per row: merged maximum and 1 / merged sum (threads t < rows); the loads of four
+          // per row: merged maximum and 1 / merged sum (threads tid < rows); the loads of four
           // pieces are in flight at once
           float *Ms = pmax_buf, *Li = lsum_buf;
-          if (t < m.rows) {
+          if (tid < m.rows) {
             float M = -INFINITY, L = 0.f;
             for (int c4 = c_first; c4 <= c_last; c4 += 4) {
               float mp[4], lp[4];
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
                 const int cc = min(c4 + k, c_last);
-                const float *Pp = P0 + (size_t)partial_slot(cc, s0, W) * pstride + (size_t)t * kPS;
+                const float *Pp = P0 + (size_t)partial_slot(cc, s0, W) * pstride + (size_t)tid * kPS;
                 mp[k] = __ldcg(Pp + kD);
                 lp[k] = __ldcg(Pp + kD + 1);
               }
@@ -729,14 +754,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
                 }
               }
             }
-            Ms[t] = M;
-            Li[t] = 1.f / L;
+            Ms[tid] = M;
+            Li[tid] = 1.f / L;
           }
           ptx::named_bar_sync(2, kSoftmaxThreads);
           // items (row, float4 column): this thread's items of a group of 8 accumulate piece by
           // piece, each piece's loads for the group in flight together
           const int nitems = m.rows * (kD / 4);
-          for (int it0 = t; it0 < nitems; it0 += 8 * kSoftmaxThreads) {
+          for (int it0 = tid; it0 < nitems; it0 += 8 * kSoftmaxThreads) {
             float4 acc[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -772,7 +797,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
               }
             }
           }
-          if (t == 0) a.ws.counters[r * a.Hkv + g] = 0;
+          if (tid == 0) a.ws.counters[r * a.Hkv + g] = 0;
         }
         ptx::named_bar_sync(2, kSoftmaxThreads);
       }
@@ -785,7 +810,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
     }
   }
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
