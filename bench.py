@@ -116,8 +116,8 @@ class ClockSampler:
 # capture of the bench's own command (the summary under profiles/ gives the command), keyed by the
 # SHA-1 of the kernel sources the capture ran; any change to those sources voids the figure.
 NCU_TRAFFIC = {
-    # profiles/attn_tc_kernel_qwen3-4b-64req_full.md: 630.812416 MB read + 8.406272 MB written
-    "qwen3-4b-64req": ("146bfa9d884c0e9215cd9c24ab05551fa22f240e", 639218688),
+    # profiles/attn_tc_kernel_qwen3-4b-64req_full.md: 630.802688 MB read + 7.636736 MB written
+    "qwen3-4b-64req": ("2c6d01e5a054ba5a4e41d2e618870a0462c2df41", 638439424),
 }
 
 
