@@ -266,29 +266,28 @@ def run_dspark(args, rank, world, device):
 
 
 def run_e2e(args, cfg, inp, step, layers, caches, tflat, dlog, L, world, device):
+    """The step through VerifyStep.run_from_host: every step copies its inputs from pinned host
+    memory (on a copy stream, each call waiting only for its own inputs) and reads its results
+    back."""
     stream = torch.cuda.current_stream()
     h = lambda t: t.detach().cpu().pin_memory() if t is not None else None
     host_in = dict(conf=h(inp.conf_ring), kv_len=h(inp.kv_len), t_ms=h(inp.t_ms),
-                   q=h(inp.q), kn=h(inp.k_new), vn=h(inp.v_new), tflat=h(tflat), dlog=h(dlog),
-                   dt=h(inp.draft_tokens), ua=h(inp.u_acc), ur=h(inp.u_res))
+                   q=h(inp.q), k_new=h(inp.k_new), v_new=h(inp.v_new), target_logits=h(tflat),
+                   draft_logits=h(dlog), draft_tokens=h(inp.draft_tokens), u_acc=h(inp.u_acc),
+                   u_res=h(inp.u_res))
     dev_in = {k: (torch.empty_like(v, device=device) if v is not None else None)
               for k, v in host_in.items()}
-    outs = [torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
-            for v in (step.verify_len, step.accepted_len, step.out_tokens, step.n_out)]
+    host_out = {k: torch.empty(getattr(step, k).shape, dtype=getattr(step, k).dtype,
+                               pin_memory=True)
+                for k in ("verify_len", "accepted_len", "out_tokens", "n_out")}
     h2d = sum(v.numel() * v.element_size() for v in host_in.values() if v is not None)
-    d2h = sum(v.numel() * v.element_size() for v in outs)
+    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
     attn_out = torch.empty_like(inp.q[0])
+    copy_stream = torch.cuda.Stream(device=device)
 
     def one():
-        for k, v in host_in.items():
-            if v is not None:
-                dev_in[k].copy_(v, non_blocking=True)
-        lay = [(dev_in["q"][i], dev_in["kn"][i], dev_in["vn"][i]) for i in range(cfg.layers)]
-        step.run(dev_in["conf"], inp.round_idx, dev_in["kv_len"], dev_in["t_ms"], lay, caches,
-                 inp.block_table, attn_out, dev_in["tflat"], dev_in["dlog"], dev_in["dt"],
-                 dev_in["ua"], dev_in["ur"], cfg.temperature)
-        for o, s in zip(outs, (step.verify_len, step.accepted_len, step.out_tokens, step.n_out)):
-            o.copy_(s, non_blocking=True)
+        step.run_from_host(host_in, dev_in, inp.round_idx, inp.block_table, caches, attn_out,
+                           cfg.temperature, copy_stream, host_out)
 
     for _ in range(max(1, min(args.warmup, 3))):
         one()
@@ -303,7 +302,7 @@ def run_e2e(args, cfg, inp, step, layers, caches, tflat, dlog, L, world, device)
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / n
-    ok = np.array_equal(outs[0].numpy(), L)
+    ok = np.array_equal(host_out["verify_len"].numpy(), L)
     return dict(ms=ms, h2d=h2d, d2h=d2h, ok=bool(ok))
 
 

@@ -62,6 +62,53 @@ class VerifyStep:
         _d.dspark_kv_commit(k_new, v_new, kv_pages, block_table, kv_len, self.q_offsets,
                             self.accepted_len, self.K, kv_len_out, stream)
 
+    INPUT_KEYS = ("conf", "kv_len", "t_ms", "q", "k_new", "v_new", "target_logits",
+                  "draft_logits", "draft_tokens", "u_acc", "u_res")
+
+    def run_from_host(self, host: dict, dev: dict, round_idx: int, block_table,
+                      kv_pages_per_layer, attn_out, temperature: float, copy_stream,
+                      host_out: dict | None = None) -> int:
+        """One step whose inputs arrive from (pinned) host memory.
+
+        `host` and `dev` map INPUT_KEYS to host tensors and same-shaped device buffers (q,
+        k_new, v_new stacked per layer; draft_logits may be None when greedy).  The copies run
+        on `copy_stream`, in the order the step consumes them, and every call waits only for
+        its own inputs: the schedule starts once the confidences and lengths have landed, and
+        layer i's attention overlaps the copy of layer i + 1's inputs.  The step's results
+        (verify_len, accepted_len, out_tokens, n_out) are copied into `host_out` (pinned host
+        tensors) on the current stream.  Returns the number of kernels launched."""
+        cur = torch.cuda.current_stream(self.q_offsets.device)
+        copy_stream.wait_stream(cur)  # the previous step is done with the device buffers
+        layers = dev["q"].shape[0]
+        e_sched, e_acc = torch.cuda.Event(), torch.cuda.Event()
+        e_layer = [torch.cuda.Event() for _ in range(layers)]
+        with torch.cuda.stream(copy_stream):
+            for k in ("conf", "kv_len", "t_ms"):
+                dev[k].copy_(host[k], non_blocking=True)
+            e_sched.record(copy_stream)
+            for i in range(layers):
+                for k in ("q", "k_new", "v_new"):
+                    dev[k][i].copy_(host[k][i], non_blocking=True)
+                e_layer[i].record(copy_stream)
+            for k in ("target_logits", "draft_logits", "draft_tokens", "u_acc", "u_res"):
+                if host.get(k) is not None:
+                    dev[k].copy_(host[k], non_blocking=True)
+            e_acc.record(copy_stream)
+        cur.wait_event(e_sched)
+        self.schedule(dev["conf"], round_idx, dev["kv_len"], dev["t_ms"])
+        self.plan(dev["kv_len"])
+        for i in range(layers):
+            cur.wait_event(e_layer[i])
+            self.attention(dev["q"][i], dev["k_new"][i], dev["v_new"][i], kv_pages_per_layer[i],
+                           block_table, dev["kv_len"], attn_out)
+        cur.wait_event(e_acc)
+        self.accept(dev["target_logits"], dev.get("draft_logits"), dev["draft_tokens"],
+                    dev["u_acc"], dev["u_res"], temperature)
+        if host_out is not None:
+            for k in ("verify_len", "accepted_len", "out_tokens", "n_out"):
+                host_out[k].copy_(getattr(self, k), non_blocking=True)
+        return 2 + layers + 2
+
     def capture(self, enqueue, warmup: int = 1) -> torch.cuda.CUDAGraph:
         """Capture `enqueue()` — any sequence of this object's calls on the current stream — as
         one CUDA graph (after `warmup` eager runs on the capture stream).  Every launch is sized

@@ -50,3 +50,38 @@ def test_step_matches_oracle_chain(cfg, tau):
                                     host(inp.u_acc), host(inp.u_res), tau)
     assert_accept_equal(gpu_a, ref_acc)
     assert binding().dspark_read_error() == 0
+
+
+@pytest.mark.parametrize("tau", [1.0, 0.0])
+def test_step_from_host_matches_device_resident_step(tau):
+    """run_from_host (inputs copied from pinned host memory on a copy stream, per-layer events)
+    gives the same results as the same step on device-resident inputs."""
+    cfg = QWEN3_4B.with_(R=10, V=3000, layers=3)
+    inp = build_step_inputs(cfg, "cuda", seed=4, layers=cfg.layers)
+    step = new_step(cfg)
+    L = oracle_schedule(inp)["verify_len"]
+    tflat = flat_target(inp, L)
+    dlog = inp.draft_logits if tau > 0 else None
+    caches = [inp.kv_caches[0]] * cfg.layers
+    out_a = torch.empty_like(inp.q[0])
+    step.run(inp.conf_ring, inp.round_idx, inp.kv_len, inp.t_ms,
+             [(inp.q[i], inp.k_new[i], inp.v_new[i]) for i in range(cfg.layers)], caches,
+             inp.block_table, out_a, tflat, dlog, inp.draft_tokens, inp.u_acc, inp.u_res, tau)
+    torch.cuda.synchronize()
+    want = {k: getattr(step, k).clone() for k in ("verify_len", "accepted_len", "out_tokens", "n_out")}
+    pin = lambda t: t.cpu().pin_memory() if t is not None else None
+    hst = dict(conf=pin(inp.conf_ring), kv_len=pin(inp.kv_len), t_ms=pin(inp.t_ms), q=pin(inp.q),
+               k_new=pin(inp.k_new), v_new=pin(inp.v_new), target_logits=pin(tflat),
+               draft_logits=pin(dlog), draft_tokens=pin(inp.draft_tokens), u_acc=pin(inp.u_acc),
+               u_res=pin(inp.u_res))
+    dev = {k: (torch.zeros_like(v, device="cuda") if v is not None else None) for k, v in hst.items()}
+    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in want.items()}
+    for k in want:
+        getattr(step, k).zero_()
+    out_b = torch.empty_like(inp.q[0])
+    step.run_from_host(hst, dev, inp.round_idx, inp.block_table, caches, out_b, tau,
+                       torch.cuda.Stream(), host_out)
+    torch.cuda.synchronize()
+    for k, v in want.items():
+        assert torch.equal(host_out[k], v.cpu()), k
+    assert torch.equal(out_a, out_b)   # the last layer's attention
