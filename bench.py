@@ -116,8 +116,8 @@ class ClockSampler:
 # capture of the bench's own command (the summary under profiles/ gives the command), keyed by the
 # SHA-1 of the kernel sources the capture ran; any change to those sources voids the figure.
 NCU_TRAFFIC = {
-    # profiles/attn_tc_kernel_qwen3-4b-64req_full.md: 630.802688 MB read + 7.636736 MB written
-    "qwen3-4b-64req": ("2c6d01e5a054ba5a4e41d2e618870a0462c2df41", 638439424),
+    # profiles/attn_tc_kernel_qwen3-4b-64req_full.md: 630.774528 MB read + 7.320576 MB written
+    "qwen3-4b-64req": ("5c554d6bfd18ce318a931909047739025f7123d1", 638095104),
 }
 
 

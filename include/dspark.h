@@ -346,6 +346,16 @@ int dspark_markov_draft(const void *block_logits, const void *E, const void *U, 
                         dspark_stream_t stream);
 
 /*
+ * dspark_selftest_wait_timeout — exercise the bounded in-kernel wait (no counterpart on the
+ * pages: it tests this library's failure handling).  One GPU thread waits, through the same
+ * bounded mbarrier wait the tensor-core attention kernel uses, on a barrier nothing arrives at,
+ * for limit_cycles SM cycles (1 .. about 4e9); it then records DSPARK_DERR_TIMEOUT in the error
+ * word and returns.  result int32 [2] (device): result[0] = 1 if the wait completed (it never
+ * should), result[1] = 1 if the abort flag was raised.  The context stays usable afterwards.
+ */
+int dspark_selftest_wait_timeout(long long limit_cycles, int32_t *result, dspark_stream_t stream);
+
+/*
  * dspark_read_error — synchronise `stream`, return the current device's sticky error word
  * in *host_code (HOST pointer; 0 = no error, else DSPARK_DERR_* bits) and clear it.
  * Returns DSPARK_OK, or DSPARK_ECUDA if the synchronisation or copy failed.

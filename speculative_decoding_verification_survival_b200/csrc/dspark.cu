@@ -389,6 +389,32 @@ int dspark_markov_draft(const void *block_logits, const void *E, const void *U, 
   return launch_status();
 }
 
+// One thread waits on an mbarrier that nothing arrives at, through the same bounded wait the
+// attention kernel uses, with a short limit; it must give up, record DSPARK_DERR_TIMEOUT and
+// return, leaving the context usable.
+__global__ void wait_selftest_kernel(long long limit_cycles, int32_t *result) {
+  __shared__ __align__(8) uint64_t mbar;
+  __shared__ volatile int abort_flag;
+  const uint32_t bar = ptx::smem_u32(&mbar);
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool completed = ptx::mbar_wait(bar, 0, &abort_flag, limit_cycles);
+    result[0] = completed ? 1 : 0;
+    result[1] = abort_flag;
+  }
+}
+
+int dspark_selftest_wait_timeout(long long limit_cycles, int32_t *result, dspark_stream_t stream) {
+  if (!result || limit_cycles < 1 || limit_cycles > ptx::kWaitLimitCycles) return DSPARK_EINVAL;
+  wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_cycles, result);
+  return launch_status();
+}
+
 int dspark_read_error(int32_t *host_code, dspark_stream_t stream) {
   if (!host_code) return DSPARK_EINVAL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

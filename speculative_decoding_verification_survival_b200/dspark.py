@@ -61,6 +61,7 @@ _SIGS = {
     "dspark_accept": ([_p, _p, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _f, _p, _p, _p, _p, _sz,
                        _p], _i),
     "dspark_read_error": ([ctypes.POINTER(ctypes.c_int32), _p], _i),
+    "dspark_selftest_wait_timeout": ([ctypes.c_longlong, _p, _p], _i),
     "dspark_markov_draft_workspace_bytes": ([_i, _i], _sz),
     "dspark_markov_draft": ([_p, _p, _p, _i, _p, _i, _i, _i, _f, ctypes.c_uint32, ctypes.c_uint32,
                              _p, _p, _p, _sz, _p], _i),
@@ -277,3 +278,9 @@ def dspark_markov_draft(block_logits, E, U, x0, temperature, round_idx, seed, dr
     _call("dspark_markov_draft", _ptr(block_logits), _ptr(E), _ptr(U), d, _ptr(x0), R, K, V,
           float(temperature), int(round_idx) & 0xFFFFFFFF, int(seed) & 0xFFFFFFFF,
           _ptr(draft_logits), _ptr(draft_tokens), _ptr(ws), ws.numel(), _stream(stream))
+
+
+def dspark_selftest_wait_timeout(limit_cycles: int, result, stream=None):
+    """A bounded in-kernel wait on a barrier nothing arrives at; result int32 [2] (device)."""
+    _check(result, torch.int32, "result")
+    _call("dspark_selftest_wait_timeout", int(limit_cycles), _ptr(result), _stream(stream))
