@@ -12,14 +12,17 @@
 //                          per-thread running max with float32 exp2 terms accumulated into
 //                          float64 sums (rescaled when the running max rises), then a block
 //                          merge -> (m, Z = sum exp((z - m)/tau); greedy: argmax, lowest index).
-//   accept_finalize_kernel one CTA per request: all draft positions tested at once, the accepted
-//                          prefix ends at the first failure; then the correction / bonus draw
-//                          by inverse CDF over one row pair: pass 1 sums the weights per
-//                          2048-element chunk (float64), the threshold u * Z picks the chunk,
-//                          pass 2 re-reads that chunk and scans it.
+//   accept_finalize_kernel one cluster of `ncl` CTAs per request: all draft positions tested at
+//                          once, the accepted prefix ends at the first failure; then the
+//                          correction / bonus draw by inverse CDF over one row pair: pass 1
+//                          sums the weights per 2048-element chunk (float64), each CTA of the
+//                          cluster over its own run of chunks; the chunk sums are gathered
+//                          through distributed shared memory and the threshold u * Z picks the
+//                          chunk; pass 2 re-reads that chunk and scans it, in the CTA owning it.
 #pragma once
 
 #include "common.cuh"
+#include "ptx_sm100.cuh"
 
 namespace dspark {
 
@@ -37,11 +40,21 @@ __host__ __device__ inline size_t accept_ws_bytes(int R, int K, int T_cap) {
   return ((size_t)T_cap + (size_t)R * K) * sizeof(RowStats);
 }
 
-// Dynamic shared memory of the finalize kernel: per-warp partial sums of every chunk, then the
-// chunk sums and two scalars.
+// Dynamic shared memory of the finalize kernel: per-warp partial sums of every chunk, this
+// CTA's chunk sums, the gathered chunk sums of the whole row and two scalars.
 __host__ __device__ inline size_t accept_finalize_smem(int V) {
   const size_t nch = ((size_t)V + kAccChunk - 1) / kAccChunk;
-  return ((size_t)kAccWarps * nch + nch + 2) * sizeof(double);
+  return ((size_t)kAccWarps * nch + 2 * nch + 2) * sizeof(double);
+}
+
+// The run of chunks [chunk_lo(k), chunk_lo(k + 1)) that CTA k of a cluster of ncl sums.
+__host__ __device__ inline int chunk_lo(int nch, int k, int ncl) {
+  return (int)((long long)nch * k / ncl);
+}
+__device__ __forceinline__ int chunk_owner(int nch, int ch, int ncl) {
+  int k = 0;
+  while (k + 1 < ncl && chunk_lo(nch, k + 1, ncl) <= ch) ++k;
+  return k;
 }
 
 template <typename T>
@@ -189,10 +202,12 @@ struct RowPair {
   float invZt, invZd;
   float c;
   bool residual, vec;
+  // Both probabilities are rounded before the difference (no fused multiply-add): equal rows
+  // with equal statistics then give exactly 0, so an empty residual is seen as empty.
   __device__ __forceinline__ float weight(float zt, float zd) const {
-    const float pt = exp2_sfu((zt - mt) * c) * invZt;
+    const float pt = __fmul_rn(exp2_sfu((zt - mt) * c), invZt);
     if (!residual) return pt;
-    return fmaxf(0.f, pt - exp2_sfu((zd - md) * c) * invZd);
+    return fmaxf(0.f, pt - __fmul_rn(exp2_sfu((zd - md) * c), invZd));
   }
 };
 
@@ -264,19 +279,25 @@ __device__ __forceinline__ double block_excl_scan_f64_acc(double x, double *sm) 
   return off + incl - x;
 }
 
-// Inverse-CDF draw over a row pair: smallest v with C(v) > u * C(V-1).  Pass 1 streams the row
-// (four chunks per step with every load of the step issued before any is used, per-warp partial
-// sums in shared memory, no barrier inside the loop); the threshold picks a chunk; pass 2
-// re-reads that chunk and scans it in index order.
+// Inverse-CDF draw over a row pair: smallest v with C(v) > u * C(V-1).  Pass 1 streams this
+// CTA's chunks of the row (four chunks per step with every load of the step issued before any
+// is used, per-warp partial sums in shared memory, no barrier inside the loop); the chunk sums of
+// all `ncl` CTAs of the cluster are gathered in index order, the threshold picks a chunk; pass 2
+// re-reads that chunk and scans it in index order, in the CTA that owns it.  Returns the token,
+// -1 in every CTA when the row has no mass, -2 in the CTAs that do not own the picked chunk.
+// Every CTA of the cluster calls it with the same row pair and u.
 template <typename T>
-__device__ int draw_inverse_cdf(const RowPair<T> &rp, int V, float u, double *fsm, double *sm) {
+__device__ int draw_inverse_cdf(const RowPair<T> &rp, int V, float u, double *fsm, double *sm,
+                                int rank, int ncl) {
   __shared__ int s_pick;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nch = (V + kAccChunk - 1) / kAccChunk;
   double *part = fsm;                         // [kAccWarps][nch]
-  double *chunk_sum = fsm + kAccWarps * nch;  // [nch + 2]
+  double *chunk_sum = fsm + kAccWarps * nch;  // [nch], this CTA's chunks
+  double *all_sum = chunk_sum + nch;          // [nch + 2], every chunk, then thr and base
+  const int lo = chunk_lo(nch, rank, ncl), hi = chunk_lo(nch, rank + 1, ncl);
   constexpr int kU = 4;
-  for (int ch0 = 0; ch0 < nch; ch0 += kU) {
+  for (int ch0 = lo; ch0 < hi; ch0 += kU) {
     float xt[kU][8], xd[kU][8];
     if (rp.vec) {  // V % 8 == 0, rows aligned: a group is either wholly inside or past the end
       Raw8<T> rt[kU], rd[kU];
@@ -304,7 +325,7 @@ __device__ int draw_inverse_cdf(const RowPair<T> &rp, int V, float u, double *fs
     }
 #pragma unroll
     for (int k = 0; k < kU; ++k) {
-      if (ch0 + k < nch) {
+      if (ch0 + k < hi) {
         float w[8];
         const double s = warp_sum(weights8(rp, (ch0 + k) * kAccChunk + tid * 8, V, xt[k], xd[k], w));
         if (lane == 0) part[warp * nch + ch0 + k] = s;
@@ -312,36 +333,46 @@ __device__ int draw_inverse_cdf(const RowPair<T> &rp, int V, float u, double *fs
     }
   }
   __syncthreads();
-  for (int ch = tid; ch < nch; ch += kAccThreads) {
+  for (int ch = lo + tid; ch < hi; ch += kAccThreads) {
     double t = 0.0;
     for (int w = 0; w < kAccWarps; ++w) t += part[w * nch + ch];
     chunk_sum[ch] = t;
   }
+  if (ncl > 1) {
+    ptx::cluster_sync();  // every CTA's chunk sums are written
+    for (int ch = tid; ch < nch; ch += kAccThreads)
+      all_sum[ch] = ptx::ld_dsmem_f64(chunk_sum + ch, (uint32_t)chunk_owner(nch, ch, ncl));
+    ptx::cluster_sync();  // every CTA has read them: shared memory may be rewritten, CTAs exit
+  } else {
+    __syncthreads();
+    for (int ch = tid; ch < nch; ch += kAccThreads) all_sum[ch] = chunk_sum[ch];
+  }
   __syncthreads();
   if (tid == 0) {
     double Z = 0.0;
-    for (int ch = 0; ch < nch; ++ch) Z += chunk_sum[ch];
+    for (int ch = 0; ch < nch; ++ch) Z += all_sum[ch];
     const double thr = (double)u * Z;
     double cum = 0.0;
     int pick = -1;
     double base = 0.0;
     for (int ch = 0; ch < nch; ++ch) {
-      if (chunk_sum[ch] > 0.0 && cum + chunk_sum[ch] > thr) { pick = ch; base = cum; break; }
-      cum += chunk_sum[ch];
+      if (all_sum[ch] > 0.0 && cum + all_sum[ch] > thr) { pick = ch; base = cum; break; }
+      cum += all_sum[ch];
     }
     if (pick < 0) {  // rounding put the threshold past the end: last chunk with mass
       for (int ch = nch - 1; ch >= 0; --ch)
-        if (chunk_sum[ch] > 0.0) { pick = ch; break; }
+        if (all_sum[ch] > 0.0) { pick = ch; break; }
       base = -1.0;   // marker: take the last positive element of that chunk
     }
-    chunk_sum[nch] = thr;
-    chunk_sum[nch + 1] = base;
+    all_sum[nch] = thr;
+    all_sum[nch + 1] = base;
     s_pick = pick;
   }
   __syncthreads();
   const int pick = s_pick;
   if (pick < 0) return -1;  // no mass anywhere
-  const double thr = chunk_sum[nch], base = chunk_sum[nch + 1];
+  if (chunk_owner(nch, pick, ncl) != rank) return -2;
+  const double thr = all_sum[nch], base = all_sum[nch + 1];
   const int b0 = pick * kAccChunk + tid * 8;
   float xt[8], xd[8];
   load_pair8_scalar(rp, b0, V, xt, xd);
@@ -364,11 +395,16 @@ __device__ int draw_inverse_cdf(const RowPair<T> &rp, int V, float u, double *fs
   if (found != 0x7fffffff) atomicMin(&s_found, found);
   if (lastpos >= 0) atomicMax(&s_lastpos, lastpos);
   __syncthreads();
-  return (s_found != 0x7fffffff) ? s_found : s_lastpos;
+  // the chunk had mass in pass 1 and pass 2 recomputes the same weights, so a position exists;
+  // were it missing, -3 keeps the retry decision (-1) the same in every CTA of the cluster
+  return (s_found != 0x7fffffff) ? s_found : (s_lastpos >= 0 ? s_lastpos : -3);
 }
 
-// One CTA per request: every draft position's test at once (one thread each), the accepted
-// prefix ending at the first failure, then the correction / bonus token.
+// One cluster of ncl CTAs per request (launched with cluster dimension ncl; ncl = 1 without
+// clusters, always so for GREEDY): every CTA takes every draft position's test at once (one
+// thread each) and finds the accepted prefix ending at the first failure; the CTAs then share
+// the correction / bonus draw.  CTA 0 writes the outputs except a drawn token, which the CTA
+// owning its chunk writes.
 template <typename T, bool GREEDY>
 __global__ void __launch_bounds__(kAccThreads)
 accept_finalize_kernel(const T *__restrict__ target, const T *__restrict__ draft, int V, int R,
@@ -377,24 +413,28 @@ accept_finalize_kernel(const T *__restrict__ target, const T *__restrict__ draft
                        const int32_t *__restrict__ q_offsets, const float *__restrict__ u_acc,
                        const float *__restrict__ u_res, float c,
                        const RowStats *__restrict__ stats, int32_t *__restrict__ accepted_len,
-                       int32_t *__restrict__ out_tokens, int32_t *__restrict__ n_out) {
+                       int32_t *__restrict__ out_tokens, int32_t *__restrict__ n_out, int ncl) {
   extern __shared__ double fsm[];
   __shared__ double sm[kAccWarps];
   __shared__ int s_fail;
-  const int r = blockIdx.x, tid = threadIdx.x;
+  const int r = blockIdx.x / ncl, tid = threadIdx.x;
+  const int rank = ncl > 1 ? (int)ptx::cluster_ctarank() : 0;
+  const bool lead = rank == 0;
   const int L = __ldg(verify_len + r);
   const int t0 = __ldg(q_offsets + r), t1 = __ldg(q_offsets + r + 1);
   const bool len_ok = L >= 0 && L <= K;
   const bool ok = len_ok && t1 - t0 == L + 1 && t0 >= 0 && t1 <= T_cap;
   if (tid == 0) {
-    if (!len_ok) raise_error(DSPARK_DERR_VERIFY_LEN);
-    else if (!ok) raise_error(DSPARK_DERR_OFFSETS);
+    if (lead && !len_ok) raise_error(DSPARK_DERR_VERIFY_LEN);
+    else if (lead && !ok) raise_error(DSPARK_DERR_OFFSETS);
     s_fail = ok ? L : 0;
   }
   __syncthreads();
-  if (!ok) {
-    for (int j = tid; j <= K; j += kAccThreads) out_tokens[(size_t)r * (K + 1) + j] = -1;
-    if (tid == 0) { accepted_len[r] = 0; n_out[r] = 0; }
+  if (!ok) {  // the same in every CTA of the cluster: none reaches a cluster barrier
+    if (lead) {
+      for (int j = tid; j <= K; j += kAccThreads) out_tokens[(size_t)r * (K + 1) + j] = -1;
+      if (tid == 0) { accepted_len[r] = 0; n_out[r] = 0; }
+    }
     return;
   }
   bool bad = false;
@@ -420,7 +460,7 @@ accept_finalize_kernel(const T *__restrict__ target, const T *__restrict__ draft
   }
   __syncthreads();
   const int a = s_fail;
-  if (tid == a && bad) raise_error(DSPARK_DERR_TOKEN);  // the token the chain stopped at
+  if (lead && tid == a && bad) raise_error(DSPARK_DERR_TOKEN);  // the token the chain stopped at
   int corr;
   if (GREEDY) {
     corr = stats[t0 + a].argmax;
@@ -446,20 +486,23 @@ accept_finalize_kernel(const T *__restrict__ target, const T *__restrict__ draft
     rp.vec = (V % 8 == 0) && ((reinterpret_cast<uintptr_t>(rp.t) & align) == 0) &&
              (!rp.residual || (reinterpret_cast<uintptr_t>(rp.d) & align) == 0);
     const float u = __ldg(u_res + (size_t)r * (K + 1) + a);
-    corr = draw_inverse_cdf(rp, V, u, fsm, sm);
-    if (corr < 0 && rp.residual) {  // residual empty in floating point: draw from p instead
+    corr = draw_inverse_cdf(rp, V, u, fsm, sm, rank, ncl);
+    if (corr == -1 && rp.residual) {  // residual empty in floating point: draw from p instead
       rp.residual = false;
       __syncthreads();
-      corr = draw_inverse_cdf(rp, V, u, fsm, sm);
+      corr = draw_inverse_cdf(rp, V, u, fsm, sm, rank, ncl);
     }
   }
-  for (int j = tid; j <= K; j += kAccThreads) {
-    int v = -1;
-    if (j < a) v = __ldg(draft_tokens + (size_t)r * K + j);
-    else if (j == a) v = corr;
-    out_tokens[(size_t)r * (K + 1) + j] = v;
+  // corr: the token in the CTA that drew it, -1 in every CTA when nothing could be drawn,
+  // -2 in the other CTAs
+  if ((corr >= 0 || corr == -3) && tid == 0) out_tokens[(size_t)r * (K + 1) + a] = max(corr, -1);
+  if (lead) {
+    for (int j = tid; j <= K; j += kAccThreads) {
+      if (j < a) out_tokens[(size_t)r * (K + 1) + j] = __ldg(draft_tokens + (size_t)r * K + j);
+      else if (j > a || corr == -1) out_tokens[(size_t)r * (K + 1) + j] = -1;
+    }
+    if (tid == 0) { accepted_len[r] = a; n_out[r] = a + 1; }
   }
-  if (tid == 0) { accepted_len[r] = a; n_out[r] = a + 1; }
 }
 
 }  // namespace dspark

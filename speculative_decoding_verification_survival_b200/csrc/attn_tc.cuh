@@ -374,6 +374,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       const int rg0 = is_k ? 0 : 2;
       const CUtensorMap *nmap = is_k ? &tmap_kn : &tmap_vn;
       const int nslots = is_k ? kSlotsK : kSlotsV;
+      // every cached page is read by exactly one CTA once: let it leave L2 first, so that the
+      // split-KV partials written early in the kernel are still there when they are merged
+      const uint64_t stream_policy = ptx::l2_policy_evict_first();
       int last_use[kMaxSlots];  // latest slot use that was armed (TMA or empty arrive), -1 if none
 #pragma unroll
       for (int k = 0; k < kMaxSlots; ++k) last_use[k] = -1;
@@ -397,8 +400,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
               raise_error(DSPARK_DERR_PAGE);
             }
             ptx::mbar_arrive_expect_tx(fb, kHalfPageBytes);
-            ptx::tma_load_2d(ring(rg0, slot), &tmap_kv, fb, 0, row);
-            ptx::tma_load_2d(ring(rg0 + 1, slot), &tmap_kv, fb, 64, row);
+            ptx::tma_load_2d_hint(ring(rg0, slot), &tmap_kv, fb, 0, row, stream_policy);
+            ptx::tma_load_2d_hint(ring(rg0 + 1, slot), &tmap_kv, fb, 64, row, stream_policy);
           } else if (tc.j == m.ncache && h == 0) {  // the verify tokens: 16 rows of KV head g
             ptx::mbar_arrive_expect_tx(fb, kNewHalfBytes);
             ptx::tma_load_3d(ring(rg0, slot), nmap, fb, 0, tc.g, m.t0);
@@ -731,64 +734,58 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
           const int c_first = s0 / W, c_last = (s0 + tiles - 1) / W;
           const size_t pstride = (size_t)a.rows_max * kPS;
           const float *P0 = a.ws.partials;
-          // per row: merged maximum and 1 / merged sum (threads tid < rows); the loads of four
-          // pieces are in flight at once
-          float *Ms = pmax_buf, *Li = lsum_buf;
-          if (tid < m.rows) {
-            float M = -INFINITY, L = 0.f;
-            for (int c4 = c_first; c4 <= c_last; c4 += 4) {
-              float mp[4], lp[4];
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const int cc = min(c4 + k, c_last);
-                const float *Pp = P0 + (size_t)partial_slot(cc, s0, W) * pstride + (size_t)tid * kPS;
-                mp[k] = __ldcg(Pp + kD);
-                lp[k] = __ldcg(Pp + kD + 1);
-              }
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                if (c4 + k <= c_last && mp[k] != -INFINITY) {
-                  const float Mn = fmaxf(M, mp[k]);
-                  L = L * ex2(M - Mn) + lp[k] * ex2(mp[k] - Mn);
-                  M = Mn;
-                }
-              }
-            }
-            Ms[tid] = M;
-            Li[tid] = 1.f / L;
-          }
-          ptx::named_bar_sync(2, kSoftmaxThreads);
-          // items (row, float4 column): this thread's items of a group of 8 accumulate piece by
-          // piece, each piece's loads for the group in flight together
+          // items (row, float4 column), four per thread: each item merges the pieces online,
+          // (m, l, values) of two pieces for all four items in flight at once, so that the usual
+          // split (this piece and one other) costs a single round trip
           const int nitems = m.rows * (kD / 4);
-          for (int it0 = tid; it0 < nitems; it0 += 8 * kSoftmaxThreads) {
-            float4 acc[8];
+          for (int it0 = tid; it0 < nitems; it0 += 4 * kSoftmaxThreads) {
+            float4 acc[4];
+            float Mi[4], Lsum[4];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int cc = c_first; cc <= c_last; ++cc) {
-              const float *Pp = P0 + (size_t)partial_slot(cc, s0, W) * pstride;
+            for (int k = 0; k < 4; ++k) {
+              acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+              Mi[k] = -INFINITY;
+              Lsum[k] = 0.f;
+            }
+            for (int c2 = c_first; c2 <= c_last; c2 += 2) {
+              float mp[2][4], lp[2][4];
+              float4 v[2][4];
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const int item = it0 + k * kSoftmaxThreads;
-                if (item < nitems) {
+              for (int pc = 0; pc < 2; ++pc) {
+                const float *Pp = P0 + (size_t)partial_slot(min(c2 + pc, c_last), s0, W) * pstride;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const int item = min(it0 + k * kSoftmaxThreads, nitems - 1);
                   const int row = item / (kD / 4), d4 = item % (kD / 4);
-                  const float mp = __ldcg(Pp + (size_t)row * kPS + kD);
-                  const float4 v = __ldcg(reinterpret_cast<const float4 *>(Pp + (size_t)row * kPS) + d4);
-                  const float wgt = (mp == -INFINITY) ? 0.f : ex2(mp - Ms[row]);
-                  acc[k].x = fmaf(v.x, wgt, acc[k].x);
-                  acc[k].y = fmaf(v.y, wgt, acc[k].y);
-                  acc[k].z = fmaf(v.z, wgt, acc[k].z);
-                  acc[k].w = fmaf(v.w, wgt, acc[k].w);
+                  mp[pc][k] = __ldcg(Pp + (size_t)row * kPS + kD);
+                  lp[pc][k] = __ldcg(Pp + (size_t)row * kPS + kD + 1);
+                  v[pc][k] = __ldcg(reinterpret_cast<const float4 *>(Pp + (size_t)row * kPS) + d4);
+                }
+              }
+#pragma unroll
+              for (int pc = 0; pc < 2; ++pc) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  if (c2 + pc <= c_last && mp[pc][k] != -INFINITY) {
+                    const float Mn = fmaxf(Mi[k], mp[pc][k]);
+                    const float so = ex2(Mi[k] - Mn), sp = ex2(mp[pc][k] - Mn);
+                    Lsum[k] = Lsum[k] * so + lp[pc][k] * sp;
+                    acc[k].x = acc[k].x * so + v[pc][k].x * sp;
+                    acc[k].y = acc[k].y * so + v[pc][k].y * sp;
+                    acc[k].z = acc[k].z * so + v[pc][k].z * sp;
+                    acc[k].w = acc[k].w * so + v[pc][k].w * sp;
+                    Mi[k] = Mn;
+                  }
                 }
               }
             }
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < 4; ++k) {
               const int item = it0 + k * kSoftmaxThreads;
               if (item < nitems) {
                 const int row = item / (kD / 4), d4 = item % (kD / 4);
                 const int jj = row / G, ii = row % G;
-                const float li = Li[row];
+                const float li = 1.f / Lsum[k];
                 uint2 w2;
                 w2.x = ptx::pack_bf16x2(acc[k].x * li, acc[k].y * li);
                 w2.y = ptx::pack_bf16x2(acc[k].z * li, acc[k].w * li);

@@ -1,6 +1,7 @@
 // libdspark: C ABI entry points (include/dspark.h).  Host-side validation, launch shapes and
 // dispatch; the kernels live in the included headers so that the whole library is one module
 // with one device error word.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdio>
@@ -272,6 +273,16 @@ int dspark_accept(const void *target_logits, const void *draft_logits, int dtype
   const int nrows = T_cap + R * K;
   const size_t fin_smem = accept_finalize_smem(V);
   if (fin_smem > 227 * 1024) return DSPARK_EUNSUPPORTED;
+  // CTAs per request for the draw: as many as keep the whole grid resident at two CTAs per SM
+  // (the sampled kernel's registers allow two), at most 8 (the portable cluster size), never
+  // more than the row has chunks
+  int ncl = 1;
+  if (!greedy) {
+    const int sms = sm_count();
+    if (sms <= 0) return DSPARK_ECUDA;
+    const int nch = (V + kAccChunk - 1) / kAccChunk;
+    ncl = std::max(1, std::min({8, nch, 2 * sms / R}));
+  }
   auto run = [&](auto tag) -> int {
     using T = decltype(tag);
     const T *tl = static_cast<const T *>(target_logits);
@@ -284,9 +295,22 @@ int dspark_accept(const void *target_logits, const void *draft_logits, int dtype
           cudaFuncSetAttribute(fin_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)fin_smem) != cudaSuccess)
         return DSPARK_ECUDA;
-      fin_kernel<<<R, kAccThreads, fin_smem, s>>>(tl, dl, V, R, K, T_cap, draft_tokens,
-                                                  verify_len, q_offsets, u_acc, u_res, c, st,
-                                                  accepted_len, out_tokens, n_out);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)(R * ncl));
+      cfg.blockDim = dim3(kAccThreads);
+      cfg.dynamicSmemBytes = fin_smem;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = (unsigned)ncl;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = ncl > 1 ? 1 : 0;
+      if (cudaLaunchKernelEx(&cfg, fin_kernel, tl, dl, V, R, K, T_cap, draft_tokens, verify_len,
+                             q_offsets, u_acc, u_res, c, (const RowStats *)st, accepted_len,
+                             out_tokens, n_out, ncl) != cudaSuccess)
+        return DSPARK_ECUDA;
       return launch_status();
     };
     if (greedy) return launch(accept_stats_kernel<T, true>, accept_finalize_kernel<T, true>);

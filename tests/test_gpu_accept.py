@@ -57,6 +57,47 @@ def test_edge_lengths_odd_vocab():
     _workload_accept(cfg, verify_len=np.zeros(40, int), temperature=0.9)
 
 
+@pytest.mark.parametrize("V", [151936, 20000 + 3, 4096 + 1])
+def test_draw_split_across_cluster(V):
+    # few requests over a long vocabulary: each request's draw is shared by a cluster of CTAs
+    # (8 CTAs for 75 chunks; 8 CTAs over 10 chunks, an uneven split, on the unaligned scalar
+    # path; 3 CTAs of one chunk each)
+    cfg = QWEN3_4B.with_(R=12, V=V)
+    for tau in (1.0, 0.6):
+        gpu, ref, _, _ = _workload_accept(cfg, seed=V % 7, temperature=tau)
+        assert np.all(gpu["out_tokens"][np.arange(12), gpu["accepted_len"]] >= 0)
+
+
+def test_empty_residual_falls_back_to_p_across_cluster():
+    # draft rows equal to the target rows of the same positions: p == q, every ratio is 1, so
+    # u = 1 rejects and leaves a residual that is zero everywhere; the draw then falls back to
+    # p, in the oracle and in the cluster of CTAs alike
+    cfg = QWEN3_4B.with_(R=12)
+    inp = build_step_inputs(cfg, "cuda", seed=5, layers=1)
+    verify_len = oracle_schedule(inp)["verify_len"]
+    step = new_step(cfg)
+    qo, _ = set_schedule(step, verify_len, host(inp.kv_len))
+    tflat = flat_target(inp, verify_len)
+    dl = inp.target_block[:, :cfg.K].contiguous()
+    u_acc = inp.u_acc.clone()
+    u_acc[::2, 0] = 1.0
+    gpu = gpu_accept(step, tflat, dl, inp.draft_tokens, u_acc, inp.u_res, 1.0)
+    ref = oracle_accept_chunked(tflat, dl, host(inp.draft_tokens), np.asarray(verify_len), qo,
+                                host(u_acc), host(inp.u_res), 1.0)
+    assert_accept_equal(gpu, ref)
+    assert binding().dspark_read_error() == 0
+    L = np.asarray(verify_len)
+    assert np.all(gpu["accepted_len"][::2][L[::2] > 0] == 0)   # rejected at once
+    assert np.all(gpu["accepted_len"][1::2] == L[1::2])         # every ratio 1: all accepted
+    assert np.all(gpu["out_tokens"][np.arange(12), gpu["accepted_len"]] >= 0)
+    # u = 1 sits on the acceptance threshold, so the oracle flags those requests; their draws
+    # from p are still compared wherever the draw itself is not near a boundary
+    even = (np.arange(12) % 2 == 0) & ~ref["flag_sample"]
+    assert even.sum() >= 4
+    assert np.array_equal(gpu["out_tokens"][even], ref["out_tokens"][even])
+    assert np.array_equal(gpu["accepted_len"][even], ref["accepted_len"][even])
+
+
 def _gpu_trials(tr, tau=1.0):
     d = binding()
     n = len(tr["verify_len"])
