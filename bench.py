@@ -116,8 +116,8 @@ class ClockSampler:
 # capture of the bench's own command (the summary under profiles/ gives the command), keyed by the
 # SHA-1 of the kernel sources the capture ran; any change to those sources voids the figure.
 NCU_TRAFFIC = {
-    # profiles/attn_tc_kernel_qwen3-4b-64req_full.md: 630.774528 MB read + 7.320576 MB written
-    "qwen3-4b-64req": ("5c554d6bfd18ce318a931909047739025f7123d1", 638095104),
+    # profiles/attn_tc_kernel_qwen3-4b-64req_full.md: 626.621440 MB read + 4.200960 MB written
+    "qwen3-4b-64req": ("350e83cbe27b76a4873216c14de15cb80d1d7f0f", 630822400),
 }
 
 
