@@ -573,6 +573,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       const int rpc = 128 / m.C;         // lanes per copy
       const int copy = t / rpc, rho = t % rpc;
       const bool active = m.valid && rho < m.rows;
+      // A split piece whose other pieces have all published by the time it starts (nearly every
+      // CTA's last piece: the next CTA took the segment's rest first) merges without publishing
+      // its own partial; this early read keeps the counter's latency off the epilogue.
+      const bool split = !(ta == 0 && tb == tiles);
+      int pre_count = -1;
+      if (tid == 0 && split) pre_count = ptx::ld_acquire_gpu(a.ws.counters + r * a.Hkv + g);
       SoftmaxState sm;
       sm.m_run = -INFINITY;
       sm.l_part = 0.f;
@@ -642,6 +648,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       if (m.ntiles > 0) {
         ptx::mbar_wait(bar(kBarODone, 0), (gt + m.ntiles - 1) & 1, abort_flag);
         ptx::tc_fence_after();
+      }
+      if (tid == 0 && split) {  // 2: merge at once (read after the next barrier)
+        const int pieces = (s0 + tiles - 1) / it.W - s0 / it.W + 1;
+        *s_last = (pre_count == pieces - 1) ? 2 : 0;
       }
       ptx::named_bar_sync(2, kSoftmaxThreads);
       const bool whole = (ta == 0 && tb == tiles);
@@ -721,12 +731,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       }
 
       if (!whole) {  // split segment: publish the partial, the last piece merges
-        __threadfence();
-        ptx::named_bar_sync(2, kSoftmaxThreads);
-        if (tid == 0) {
-          const int pieces = (s0 + tiles - 1) / W - s0 / W + 1;
-          const int prev = atomicAdd(a.ws.counters + r * a.Hkv + g, 1);
-          *s_last = (prev == pieces - 1);
+        if (*s_last != 2) {
+          __threadfence();
+          ptx::named_bar_sync(2, kSoftmaxThreads);
+          if (tid == 0) {
+            const int pieces = (s0 + tiles - 1) / W - s0 / W + 1;
+            const int prev = atomicAdd(a.ws.counters + r * a.Hkv + g, 1);
+            *s_last = (prev == pieces - 1);
+          }
+        } else {
+          // every other piece published before this one started (tid 0's acquire read of the
+          // counter, ordered for the CTA by the barriers): no publish, no count; the merge below
+          // reads this CTA's own partial after the barrier and resets the counter
         }
         ptx::named_bar_sync(2, kSoftmaxThreads);
         if (*s_last) {
