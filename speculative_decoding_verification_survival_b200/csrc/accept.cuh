@@ -69,9 +69,10 @@ __device__ __forceinline__ float exp2_sfu(float x) {
 
 // One CTA per scheduled logit row: one streaming pass with 16-byte loads, 32 elements per thread
 // and step; the running maximum rescales the float64 sum only when it rises.  GREEDY rows only
-// need the maximum and its lowest index.
+// need the maximum and its lowest index.  Five CTAs per SM (registers capped to fit), so that a
+// 64-request step's 704 rows run as one wave of 740 rather than 1.2 waves of 592.
 template <typename T, bool GREEDY>
-__global__ void __launch_bounds__(kAccThreads)
+__global__ void __launch_bounds__(kAccThreads, 5)
 accept_stats_kernel(const T *__restrict__ target, const T *__restrict__ draft, int V, int R, int K,
                     int T_cap, const int32_t *__restrict__ verify_len,
                     const int32_t *__restrict__ q_offsets, float c,
