@@ -116,8 +116,8 @@ class ClockSampler:
 # capture of the bench's own command (the summary under profiles/ gives the command), keyed by the
 # SHA-1 of the kernel sources the capture ran; any change to those sources voids the figure.
 NCU_TRAFFIC = {
-    # profiles/attn_tc_kernel_qwen3-4b-64req_full.md: 626.621440 MB read + 4.200960 MB written
-    "qwen3-4b-64req": ("350e83cbe27b76a4873216c14de15cb80d1d7f0f", 630822400),
+    # profiles/attn_tc_kernel_qwen3-4b-64req_full.md: 626.618624 MB read + 4.616192 MB written
+    "qwen3-4b-64req": ("b7667a45921c3d9cfd3c89a9121bfc2c701ef656", 631234816),
 }
 
 
