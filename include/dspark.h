@@ -207,9 +207,17 @@ size_t dspark_accept_workspace_bytes(int R, int K, int T_cap);
  *       u_acc[r][k] < min(1, p_k(x_k) / q_k(x_k));
  *   a = accepted count before the first rejection;
  *   a < L : correction drawn from max(0, p_a - q_a) (normalised), a == L: bonus from p_L;
- *   draw = smallest v with C(v) > u_res[r][a] * C(V-1), C the running sum in index order.
+ *   draw = smallest v with C(v) > u_res[r][a] * C(V-1), C the running sum in index order;
+ *   a residual that is empty in floating point (p_a <= q_a everywhere, e.g. a draft row equal
+ *   to its target row) falls back to a draw from p_a.
  * temperature <= 0 selects greedy verification: accept iff x_k == argmax of target row k
  * (lowest index on ties); the correction / bonus is the argmax of target row a.
+ * u_acc = 1 rejects at any ratio.
+ *
+ * Launches: one CTA per scheduled logit row for the statistics, then the finalize kernel.
+ * In sampled mode the finalize kernel runs a thread-block cluster of up to 8 CTAs per request,
+ * which share the draw through distributed shared memory; in greedy mode it runs one CTA per
+ * request.  The result does not depend on the cluster size.
  *
  * target_logits [T_cap][V] (row q_offsets[r] + j = position j+1 of request r),
  * draft_logits [R][K][V], dtype DSPARK_BF16 or DSPARK_F32; draft_tokens int32 [R][K];
