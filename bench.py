@@ -157,6 +157,46 @@ def logits_bytes(verify_len, cfg, greedy):
     return rows * cfg.V * esz
 
 
+REJECT_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def clocks_rejected(summary):
+    """Why a timed run's clock record rejects it, or None when it stands.  A run is rejected
+    when it saw a hardware or thermal slowdown, or when its SM clock stayed well below the
+    maximum with no reason active (a leftover clock lock).  sw_power_cap alone is kept."""
+    if not summary or "sm_mhz" not in summary:
+        return None
+    bad = [r for r in summary.get("reasons", []) if r in REJECT_REASONS]
+    if bad:
+        return "+".join(bad)
+    if not summary.get("reasons") and summary["sm_mhz"] < 0.75 * summary["sm_max_mhz"]:
+        return "SM clock held below 0.75 of max with no reason active"
+    return None
+
+
+def agree_any(flag, device, world):
+    """True on every rank when `flag` is true on any rank (so that all ranks take the same
+    collective steps)."""
+    if world == 1:
+        return bool(flag)
+    t = torch.tensor([int(bool(flag))], dtype=torch.int32, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return bool(t.item())
+
+
+def measure_with_retry(timed, agree):
+    """timed() -> (result, clocks).  When the clock record of the run rejects it on any rank,
+    every rank measures once more and keeps the second result; the first run's clocks and the
+    reason are kept under clocks["first_run"]."""
+    res, clocks = timed()
+    why = clocks_rejected(clocks)
+    if agree(why is not None):
+        first = dict(clocks or {}, rejected=why or "another rank's clock record")
+        res, clocks = timed()
+        clocks = dict(clocks, first_run=first) if clocks else {"first_run": first}
+    return res, clocks
+
+
 def kv_copies_for(cfg, kv_bytes_per_layer, layers):
     """Distinct KV caches to rotate through so that one layer call never finds the previous
     call's KV in the 126 MB L2 (at least 4x L2 between reuses)."""
@@ -235,19 +275,25 @@ def run_dspark(args, rank, world, device):
     graph = step.capture(timed_steps, warmup=0)
     graph.replay()          # first replay uploads the graph; untimed
     torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        torch.cuda.synchronize()
+
+    def timed_replay():
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            torch.cuda.synchronize()
+            if world > 1:
+                torch.distributed.barrier()
+            t0.record(stream)
+            graph.replay()
+            t1.record(stream)
+            torch.cuda.synchronize()
         if world > 1:
             torch.distributed.barrier()
-        t0.record(stream)
-        graph.replay()
-        t1.record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    ms_total = t0.elapsed_time(t1)
-    attn_ms = [ev[0].elapsed_time(ev[1]) / cfg.layers for ev in ev_attn]
+        attn = [ev[0].elapsed_time(ev[1]) / cfg.layers for ev in ev_attn]
+        return (t0.elapsed_time(t1), attn), clk.summary()
+
+    # a run whose clock record shows a slowdown (or a leftover clock lock) is measured again
+    (ms_total, attn_ms), clocks = measure_with_retry(
+        timed_replay, lambda flag: agree_any(flag, device, world))
     del graph
 
     # end to end through the public step API with host buffers (pinned), copies inside
@@ -258,7 +304,7 @@ def run_dspark(args, rank, world, device):
     acc = step.accepted_len.cpu().numpy()
     res = dict(ms_total=ms_total, attn_ms=float(np.mean(attn_ms)), L=L, kv_len=kv_len, acc=acc,
                ms_eager=ms_eager, draft_ms=draft_ms,
-               clocks=clk.summary(), launches=launches_per_step * args.steps, e2e=e2e,
+               clocks=clocks, launches=launches_per_step * args.steps, e2e=e2e,
                attn_bytes=attn_bytes(kv_len, L, cfg),
                step_bytes=cfg.layers * attn_bytes(kv_len, L, cfg) + logits_bytes(L, cfg, greedy),
                kv_copies=copies)
