@@ -265,3 +265,25 @@ def test_zero_uniform_picks_first_positive_mass():
     res = _run(tr)
     assert np.all(res["accepted_len"][:32] == 0) and np.all(res["out_tokens"][:32, 0] == 2)
     assert np.all(res["accepted_len"][32:] == 2) and np.all(res["out_tokens"][32:, 2] == 2)
+
+
+def test_empty_residual_draws_from_target():
+    """p == q with u = 1 rejects the first draft token and leaves max(0, p - q) = 0 everywhere;
+    the correction is then drawn from p by the same inverse CDF (hand-computed cumulative
+    boundaries 0.1, 0.3, 0.6 of p = (0.1, 0.2, 0.3, 0.4)), and over many trials it follows p."""
+    p = [0.1, 0.2, 0.3, 0.4]
+    z = logits_of(p)
+    zt = np.tile(z, (K + 1, 1))
+    zd = np.tile(z, (K, 1))
+    rng = np.random.default_rng(17)
+    tr = build_trials(zt, zd, 3, 200_000, rng, round_idx=4)
+    tr["u_acc"] = np.array(tr["u_acc"], copy=True)
+    tr["u_res"] = np.array(tr["u_res"], copy=True)
+    tr["u_acc"][:, 0] = 1.0
+    tr["u_res"][:4, 0] = [0.05, 0.15, 0.45, 0.95]
+    res = _run(tr)
+    assert np.all(res["accepted_len"] == 0)
+    assert np.all(res["n_out"] == 1)
+    assert res["out_tokens"][:4, 0].tolist() == [0, 1, 2, 3]
+    assert np.all(res["out_tokens"][:, 1:] == -1)
+    _chi2_ok(np.bincount(res["out_tokens"][:, 0], minlength=4), target_probs(z))
