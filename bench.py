@@ -157,6 +157,17 @@ def logits_bytes(verify_len, cfg, greedy):
     return rows * cfg.V * esz
 
 
+def logits_bytes_strict(verify_len, accepted_len, cfg, greedy):
+    """The logit bytes a step must read at the least: per request the target rows of positions
+    1..a+1 and, unless greedy, the draft rows of positions 1..min(a+1, L), i.e. the rows up to
+    and including the first rejection (or the bonus row); the rest of the block is never used."""
+    esz = 2 if cfg.dtype == "bf16" else 4
+    L = np.asarray(verify_len, np.int64)
+    a = np.asarray(accepted_len, np.int64)
+    rows = int((a + 1).sum()) + (0 if greedy else int(np.minimum(a + 1, L).sum()))
+    return rows * cfg.V * esz
+
+
 REJECT_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
 
@@ -307,6 +318,8 @@ def run_dspark(args, rank, world, device):
                clocks=clocks, launches=launches_per_step * args.steps, e2e=e2e,
                attn_bytes=attn_bytes(kv_len, L, cfg),
                step_bytes=cfg.layers * attn_bytes(kv_len, L, cfg) + logits_bytes(L, cfg, greedy),
+               step_bytes_strict=cfg.layers * attn_bytes(kv_len, L, cfg)
+               + logits_bytes_strict(L, acc, cfg, greedy),
                kv_copies=copies)
     return cfg, res
 
@@ -521,6 +534,11 @@ def main():
             mean_verify_len=L_tot / R_tot, mean_accepted=acc_tot / R_tot,
             step_hbm_gbs=step_gbs, step_frac_of_8tbs=step_gbs / 8000.0,
             step_frac_of_measured=step_gbs / peak,
+            strict_lower_bound=dict(
+                bytes_per_step=res["step_bytes_strict"],
+                hbm_gbs=res["step_bytes_strict"] / (ms_step * 1e-3) / 1e9,
+                frac_of_measured=res["step_bytes_strict"] / (ms_step * 1e-3) / 1e9 / peak,
+                rows="logit rows only up to each request's first rejection"),
             roofline=dict(bound="hbm", kernel="dspark_verify_attn", achieved=achieved, peak=peak,
                           unit="GB/s", frac=achieved / peak,
                           traffic=measured_traffic(cfg.name),

@@ -1,7 +1,8 @@
 """bench.py's clock record on the host: parsing of the sampled nvidia-smi lines, which runs it
 rejects (hardware or thermal slowdown, or an SM clock held low with no reason active; the power
 cap alone is kept), and the one re-measurement, agreed by every rank so that all of them take
-the same collective steps (two `gloo` ranks)."""
+the same collective steps (two `gloo` ranks); and the strict lower bound on a step's logit bytes
+(rows up to each request's first rejection)."""
 import datetime
 import os
 import socket
@@ -106,3 +107,24 @@ def test_retry_is_agreed_by_every_rank():
     # rank 1 saw a slowdown: both ranks measured twice and kept the second run
     assert res[1] == (2, 2, "hw_slowdown")
     assert res[0] == (2, 2, "another rank's clock record")
+
+
+def test_strict_lower_bound_counts_rows_up_to_the_first_rejection():
+    from workloads.configs import TINY
+    cfg = TINY.with_(V=10, dtype="bf16")
+    L, a = [5, 0, 3], [2, 0, 3]
+    # target rows 3 + 1 + 4, draft rows min(3, 5) + min(1, 0) + min(4, 3) = 3 + 0 + 3
+    assert bench.logits_bytes_strict(L, a, cfg, greedy=False) == (8 + 6) * 10 * 2
+    assert bench.logits_bytes_strict(L, a, cfg, greedy=True) == 8 * 10 * 2
+    # every scheduled row: target 6 + 1 + 4, draft 5 + 0 + 3
+    assert bench.logits_bytes(L, cfg, greedy=False) == (11 + 8) * 10 * 2
+    import numpy as np
+    rng = np.random.default_rng(0)
+    for _ in range(100):
+        Lr = rng.integers(0, 6, size=16)
+        ar = rng.integers(0, Lr + 1)
+        for g in (False, True):
+            assert bench.logits_bytes_strict(Lr, ar, cfg, g) <= bench.logits_bytes(Lr, cfg, g)
+            if not g and np.all(ar == Lr):
+                # all accepted: every draft row plus one extra target row per request is read
+                assert bench.logits_bytes_strict(Lr, ar, cfg, g) == bench.logits_bytes(Lr, cfg, g)
