@@ -59,7 +59,10 @@ enum dspark_status {
   DSPARK_ECUDA = -2,         /* a CUDA runtime call failed (launch, attribute, copy) */
   DSPARK_EWORKSPACE = -3,    /* workspace NULL or smaller than the size query returned */
   DSPARK_EDEVICE_DATA = -4,  /* dspark_read_error: device-resident data was invalid */
-  DSPARK_ETIMEOUT = -5,      /* reserved for bounded waits; no current kernel waits */
+  DSPARK_ETIMEOUT = -5,      /* not returned by any entry point: an in-kernel wait that runs
+                                out (the tensor-core attention kernel bounds every wait at
+                                about 2 s) is reported as DSPARK_DERR_TIMEOUT in the device
+                                error word instead, because kernels return no status */
   DSPARK_EUNSUPPORTED = -6   /* valid arguments outside what this build implements */
 };
 
@@ -249,7 +252,9 @@ int dspark_accept(const void *target_logits, const void *draft_logits, int dtype
  * DSPARK_EUNSUPPORTED before anything is enqueued.  The array (16 bytes per row, 1 MiB) is held
  * by every GPU that loads the library until the process exits.
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress)
- * with that device current; make that first call before any stream capture.
+ * with that device current, and so does the first call after the device's context was
+ * recreated (cudaDeviceReset moves the array); make such a first call before any stream
+ * capture.
  * All calls on a device share the one array and it keeps the previous call's contents (every
  * row a call reads is written by that call first).  Calls whose executions overlap on the GPU
  * — on different streams, or from different host threads — race on the array: serialise them.

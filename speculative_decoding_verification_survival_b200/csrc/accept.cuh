@@ -12,6 +12,9 @@
 //                          per-thread running max with float32 exp2 terms accumulated into
 //                          float64 sums (rescaled when the running max rises), then a block
 //                          merge -> (m, Z = sum exp((z - m)/tau); greedy: argmax, lowest index).
+//                          The exponent (z - m) log2(e) / tau is formed with log2(e) / tau split
+//                          into two floats, so that the rounding of that constant (the same in
+//                          every term, hence not averaged out) does not bias Z.
 //   accept_finalize_kernel one cluster of `ncl` CTAs per request: all draft positions tested at
 //                          once, the accepted prefix ends at the first failure; then the
 //                          correction / bonus draw by inverse CDF over one row pair: pass 1
@@ -67,6 +70,20 @@ __device__ __forceinline__ float exp2_sfu(float x) {
   return y;
 }
 
+// The scale c = log2(e) / tau as an unevaluated float sum hi + lo (lo = c - hi rounded), and in
+// float64 for the few per-request evaluations done at that precision.
+struct ExpScale {
+  float hi, lo;
+  double d;
+  // d * c in float32 without the systematic error of a rounded c.  d = -inf (a masked logit,
+  // or padding) is first clamped to a large finite negative number, whose 2^x is still 0:
+  // -inf * lo would give NaN when lo is 0 or has the opposite sign of hi.
+  __device__ __forceinline__ float mul(float d_) const {
+    d_ = fmaxf(d_, -1e30f);
+    return fmaf(d_, lo, d_ * hi);
+  }
+};
+
 // One CTA per scheduled logit row: one streaming pass with 16-byte loads, 32 elements per thread
 // and step; the running maximum rescales the float64 sum only when it rises.  GREEDY rows only
 // need the maximum and its lowest index.  Five CTAs per SM (registers capped to fit), so that a
@@ -75,7 +92,7 @@ template <typename T, bool GREEDY>
 __global__ void __launch_bounds__(kAccThreads, 5)
 accept_stats_kernel(const T *__restrict__ target, const T *__restrict__ draft, int V, int R, int K,
                     int T_cap, const int32_t *__restrict__ verify_len,
-                    const int32_t *__restrict__ q_offsets, float c,
+                    const int32_t *__restrict__ q_offsets, ExpScale c,
                     RowStats *__restrict__ stats) {
   const int b = blockIdx.x;
   const T *row;
@@ -109,7 +126,7 @@ accept_stats_kernel(const T *__restrict__ target, const T *__restrict__ draft, i
 #pragma unroll
         for (int e = 0; e < 8; ++e) lm = fmaxf(lm, x[u][e]);
       if (lm > m) {
-        if (m != -INFINITY) Z *= exp2((double)(m - lm) * (double)c);
+        if (m != -INFINITY) Z *= exp2(((double)m - (double)lm) * c.d);
         m = lm;
       }
       if (m != -INFINITY) {
@@ -118,8 +135,8 @@ accept_stats_kernel(const T *__restrict__ target, const T *__restrict__ draft, i
         for (int u = 0; u < 4; ++u)
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
-            s0 += exp2_sfu((x[u][e] - m) * c);
-            s1 += exp2_sfu((x[u][e + 1] - m) * c);
+            s0 += exp2_sfu(c.mul(x[u][e] - m));
+            s1 += exp2_sfu(c.mul(x[u][e + 1] - m));
           }
         Z += (double)(s0 + s1);
       }
@@ -175,8 +192,9 @@ accept_stats_kernel(const T *__restrict__ target, const T *__restrict__ draft, i
   int I = 0x7fffffff;
   for (int w = 0; w < kAccWarps; ++w)
     if (sm_m[w] == M) I = min(I, sm_i[w]);
-  double z = (!GREEDY && m != -INFINITY && M != -INFINITY) ? Z * exp2((double)(m - M) * (double)c)
-                                                           : 0.0;
+  double z = (!GREEDY && m != -INFINITY && M != -INFINITY)
+                 ? Z * exp2(((double)m - (double)M) * c.d)
+                 : 0.0;
   z = warp_sum(z);
   if (lane == 0) sm_z[warp] = z;
   __syncthreads();
@@ -201,14 +219,14 @@ struct RowPair {
   const T *d;  // draft row (residual only)
   float mt, md;
   float invZt, invZd;
-  float c;
+  ExpScale c;
   bool residual, vec;
   // Both probabilities are rounded before the difference (no fused multiply-add): equal rows
   // with equal statistics then give exactly 0, so an empty residual is seen as empty.
   __device__ __forceinline__ float weight(float zt, float zd) const {
-    const float pt = __fmul_rn(exp2_sfu((zt - mt) * c), invZt);
+    const float pt = __fmul_rn(exp2_sfu(c.mul(zt - mt)), invZt);
     if (!residual) return pt;
-    return fmaxf(0.f, pt - __fmul_rn(exp2_sfu((zd - md) * c), invZd));
+    return fmaxf(0.f, pt - __fmul_rn(exp2_sfu(c.mul(zd - md)), invZd));
   }
 };
 
@@ -412,7 +430,7 @@ accept_finalize_kernel(const T *__restrict__ target, const T *__restrict__ draft
                        int K, int T_cap, const int32_t *__restrict__ draft_tokens,
                        const int32_t *__restrict__ verify_len,
                        const int32_t *__restrict__ q_offsets, const float *__restrict__ u_acc,
-                       const float *__restrict__ u_res, float c,
+                       const float *__restrict__ u_res, ExpScale c,
                        const RowStats *__restrict__ stats, int32_t *__restrict__ accepted_len,
                        int32_t *__restrict__ out_tokens, int32_t *__restrict__ n_out, int ncl) {
   extern __shared__ double fsm[];
@@ -451,8 +469,10 @@ accept_finalize_kernel(const T *__restrict__ target, const T *__restrict__ draft
         const RowStats sd = stats[T_cap + r * K + tid];
         const float zt = ld1(target + (size_t)(t0 + tid) * V + x);
         const float zd = ld1(draft + ((size_t)r * K + tid) * V + x);
-        const double p = (double)exp2_sfu((zt - st.m) * c) / st.Z;
-        const double q = (double)exp2_sfu((zd - sd.m) * c) / sd.Z;
+        // p(x) and q(x) in float64: a draft token far below its row's maximum has an exponent
+        // of 30-40 whose float32 evaluation would be off by more than the 1e-6 decision window
+        const double p = exp2(((double)zt - (double)st.m) * c.d) / st.Z;
+        const double q = exp2(((double)zd - (double)sd.m) * c.d) / sd.Z;
         const double ratio = (q > 0.0) ? p / q : (p > 0.0 ? INFINITY : 0.0);
         fail = !((double)__ldg(u_acc + (size_t)r * K + tid) < fmin(1.0, ratio));
       }

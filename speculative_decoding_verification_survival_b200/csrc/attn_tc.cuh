@@ -75,7 +75,7 @@ constexpr int kPS = part_stride(kD);                 // floats per split-KV part
 // aux region layout (bytes)
 constexpr uint32_t kBarKFull = 0, kBarVFull = 64, kBarKEmpty = 128, kBarVEmpty = 192,
                    kBarSFull = 256, kBarPFull = 272, kBarODone = 280, kBarQFull = 288,
-                   kBarQEmpty = 296, kBarOFree = 304;
+                   kBarQEmpty = 296, kBarOFree = 304, kBarDrain = 312;
 constexpr uint32_t kAuxTmem = 320, kAuxAbort = 324, kAuxLast = 328, kAuxPmax = 512,
                    kAuxLsum = 512 + 2 * kSoftmaxThreads * 4;
 
@@ -336,6 +336,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
     ptx::mbar_init(bar(kBarQFull, 0), kSoftmaxThreads);
     ptx::mbar_init(bar(kBarQEmpty, 0), 1);
     ptx::mbar_init(bar(kBarOFree, 0), kSoftmaxThreads);
+    ptx::mbar_init(bar(kBarDrain, 0), 1);
     *abort_flag = 0;
     *s_last = 0;
     ptx::fence_mbar_init();
@@ -497,9 +498,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
           raise_error(DSPARK_DERR_TIMEOUT);
         }
       }
-      if (cp.gt > 0 && !*abort_flag) {  // every MMA of this CTA has completed before TMEM is released
+      // Every MMA this thread issued has completed before the CTA releases its shared memory
+      // and TMEM, also after an abort (which can leave S MMAs issued after the last P.V): one
+      // more commit tracks all of them, and its wait is bounded but ignores the abort flag.
+      if (cs.gt > 0 || cp.gt > 0) {
+        ptx::mma_commit(bar(kBarDrain, 0));
         volatile int no_abort = 0;
-        ptx::mbar_wait(bar(kBarODone, 0), (cp.gt - 1) & 1, &no_abort);
+        ptx::mbar_wait(bar(kBarDrain, 0), 0, &no_abort);
       }
     }
   } else {

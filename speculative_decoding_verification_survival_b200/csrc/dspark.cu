@@ -3,6 +3,7 @@
 // with one device error word.
 #include <algorithm>
 #include <atomic>
+#include <mutex>
 #include <cmath>
 #include <cstdio>
 
@@ -267,7 +268,10 @@ int dspark_accept(const void *target_logits, const void *draft_logits, int dtype
   if (V < 1 || R < 1 || K < 1 || K > DSPARK_MAX_K || T_cap < R) return DSPARK_EINVAL;
   if (dtype != DSPARK_BF16 && dtype != DSPARK_F32) return DSPARK_EINVAL;
   if (!ws || ws_bytes < accept_ws_bytes(R, K, T_cap) || !aligned16(ws)) return DSPARK_EWORKSPACE;
-  const float c = greedy ? 0.f : (float)(1.4426950408889634 / (double)temperature);
+  ExpScale c;
+  c.d = greedy ? 0.0 : 1.4426950408889634 / (double)temperature;
+  c.hi = (float)c.d;
+  c.lo = (float)(c.d - (double)c.hi);
   RowStats *st = static_cast<RowStats *>(ws);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int nrows = T_cap + R * K;
@@ -460,13 +464,46 @@ int dspark_read_error(int32_t *host_code, dspark_stream_t stream) {
 // runtime forbids allocation after start-up, or an allocation's implicit synchronisation is not
 // acceptable).  The per-row statistics the acceptance kernels need live in this fixed array
 // instead of a caller workspace.  In host code `g_accept_noalloc_scratch` only names the
-// symbol; its device address is looked up once per device (with that device current) and that
-// address is what the kernels receive.
+// symbol; its device address is looked up once per device and context (with that device
+// current) and that address is what the kernels receive.
 static __device__ __align__(256) RowStats g_accept_noalloc_scratch[DSPARK_ACCEPT_NOALLOC_MAX_ROWS];
 
 namespace {
 constexpr int kNoAllocMaxDevices = 64;
-std::atomic<void *> g_noalloc_scratch_addr[kNoAllocMaxDevices];
+
+// The array's device address belongs to the context that loaded this module.  A device reset
+// (cudaDeviceReset, or the primary context released and created again) loads the module anew
+// and may place the array elsewhere, so the cached address is kept together with the id of the
+// context it was looked up in and looked up again when the current context's id differs.
+struct NoAllocScratch {
+  unsigned long long ctx_id = 0;  // 0: not looked up yet
+  void *addr = nullptr;
+};
+NoAllocScratch g_noalloc_scratch[kNoAllocMaxDevices];
+std::mutex g_noalloc_mutex;
+
+// Unique id of the calling thread's current context (driver entry points through the runtime,
+// no link-time libcuda); false if it cannot be read.
+bool current_context_id(unsigned long long *id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
 }  // namespace
 
 extern "C" int dspark_accept_noalloc(const void *target_logits, const void *draft_logits,
@@ -481,11 +518,22 @@ extern "C" int dspark_accept_noalloc(const void *target_logits, const void *draf
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DSPARK_ECUDA;
   if (dev < 0 || dev >= kNoAllocMaxDevices) return DSPARK_EUNSUPPORTED;
-  void *scratch = g_noalloc_scratch_addr[dev].load(std::memory_order_acquire);
-  if (scratch == nullptr) {
-    if (cudaGetSymbolAddress(&scratch, g_accept_noalloc_scratch) != cudaSuccess || !scratch)
-      return DSPARK_ECUDA;
-    g_noalloc_scratch_addr[dev].store(scratch, std::memory_order_release);
+  void *scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    NoAllocScratch &e = g_noalloc_scratch[dev];
+    unsigned long long ctx_id = 0;
+    // no current context yet: the symbol lookup below makes the runtime create it
+    const bool have_ctx = current_context_id(&ctx_id);
+    if (!have_ctx || e.ctx_id != ctx_id || e.addr == nullptr) {
+      void *p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_accept_noalloc_scratch) != cudaSuccess || !p)
+        return DSPARK_ECUDA;
+      if (!have_ctx && !current_context_id(&ctx_id)) return DSPARK_ECUDA;
+      e.addr = p;
+      e.ctx_id = ctx_id;
+    }
+    scratch = e.addr;
   }
   return dspark_accept(target_logits, draft_logits, dtype, V, R, K, T_cap, draft_tokens,
                        verify_len, q_offsets, u_acc, u_res, temperature, accepted_len,
