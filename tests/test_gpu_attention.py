@@ -2,7 +2,9 @@
 
 Small cases compare every output element (several 64-key tiles, ragged tails, empty caches,
 zero-length schedules, page crossings, all GQA group sizes used by the workloads); the full
-workloads compare sampled (token, head) rows computed one by one by the oracle.
+workloads compare sampled (token, head) rows computed one by one by the oracle (every row when
+the workload has few verify tokens), and every output element against a closed form on
+structured keys and values that make any misrouted page, head, d-half or split piece visible.
 """
 import math
 
@@ -13,6 +15,7 @@ import torch
 import oracle
 from tests.gpu_support import (ATTN_MAX_ABS, ATTN_MEAN_ABS, F32_ATTN_MAX_ABS, binding, host,
                                new_step, oracle_attn_rows, set_schedule)
+from tests.structured_attn import install_structured, structured_expected
 from workloads.configs import CONFIGS, TINY, QWEN3_4B
 from workloads.generate import build_step_inputs
 
@@ -99,6 +102,8 @@ def test_full_workload_sampled_rows(name):
     r_long = int(np.argmax(kv))
     toks |= {int(qo[r_long]), int(qo[r_long + 1]) - 1}
     rows = [(t, int(rng.integers(0, cfg.Hq))) for t in sorted(toks)]
+    if T * cfg.Hq <= 4096:   # few verify tokens (sweep-1req: one request cut into many pieces)
+        rows = [(t, h) for t in range(T) for h in range(cfg.Hq)]
     ref = oracle_attn_rows(inp, 0, inp.kv_caches[0], qo, mk, rows, step.scale)
     errs = np.concatenate([np.abs(host(out[t, h]).astype(np.float64) - ref[(t, h)])
                            for t, h in rows])
@@ -208,3 +213,26 @@ def test_tensor_core_rescale_path():
 def test_tensor_core_pages_of_128():
     cfg = QWEN3_4B.with_(R=5, page_size=128, kv_dist=("uniform", 1, 1000), V=64)
     _compare_with_scale(cfg, np.array([5, 4, 3, 2, 1]), seed=6, scale=1.0 / math.sqrt(128))
+
+
+@pytest.mark.parametrize("name", ["qwen3-4b-64req", "lognormal-1024req", "mixed-256req",
+                                  "sweep-1req", "sweep-2048req"])
+def test_full_workload_structured_keys_and_values(name):
+    cfg = CONFIGS[name]
+    inp = build_step_inputs(cfg, "cuda", seed=0, layers=1)
+    install_structured(inp)
+    step = new_step(cfg)
+    kv = host(inp.kv_len).astype(np.int64)
+    sref = oracle.schedule_ref(inp.conf_history[oracle.lagged_round(inp.round_idx)], kv,
+                               host(inp.t_ms), cfg.T_cap)
+    qo, mk = set_schedule(step, sref["verify_len"], kv)
+    out = _run_attn(step, inp)
+    T = int(qo[-1])
+    ref = structured_expected(inp, qo, kv)                    # [T][Hkv][D]
+    got = host(out[:T]).astype(np.float64).reshape(T, cfg.Hkv, cfg.G, cfg.D)
+    err = np.abs(got - ref[:, :, None, :])
+    bound = 2.0 ** -8 * np.abs(ref)[:, :, None, :] + 1e-5     # the final bf16 rounding
+    bad = err > bound
+    assert not bad.any(), (f"{int(bad.sum())} of {bad.size} elements off, worst "
+                           f"{float((err - bound).max()):.3e} at {np.argwhere(bad)[0].tolist()}")
+    assert binding().dspark_read_error() == 0

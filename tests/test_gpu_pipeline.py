@@ -1,11 +1,13 @@
-"""Verify rounds as CUDA-graph replays (pipeline.RoundPipeline) against the same rounds run
-eagerly: bit-identical outputs round after round, with the committed cache lengths and pages
-carried on the device; plus a whole step captured with VerifyStep.capture."""
+"""Verify rounds as CUDA-graph replays (pipeline.RoundPipeline): against the oracle chain
+(schedule on the lagged confidences, attention per layer, acceptance, KV commit, committed
+lengths carried forward), and against the same rounds run eagerly (bit-identical outputs round
+after round, with the committed cache lengths and pages carried on the device); plus a whole
+step captured with VerifyStep.capture."""
 import numpy as np
 import pytest
 import torch
 
-from tests.gpu_support import binding, host, new_step
+from tests.gpu_support import assert_accept_equal, binding, host, new_step
 from workloads.configs import QWEN3_4B
 from workloads.generate import build_step_inputs, flatten_target
 
@@ -95,3 +97,73 @@ def test_captured_step_replays_the_eager_step():
     got = outs + [step.accepted_len, step.out_tokens]
     for a, b in zip(ref, got):
         assert torch.equal(a, b)
+
+
+def test_graph_rounds_follow_the_oracle_chain():
+    """Five rounds replayed as CUDA graphs, each checked against the oracle chain run on the
+    same input bits: schedule_ref on the confidences of two rounds earlier, attn_ref_flat per
+    layer over the oracle's own cache, accept_ref, kv_commit_ref, and the committed lengths
+    carried into the next round.  Lengths, markers and tokens are bit-exact (a request the
+    oracle flags may differ; the chain then continues from the GPU's decision, the only other
+    valid one), attention is within the stated bf16 tolerance and the caches are byte-exact."""
+    import math
+
+    import oracle
+    from tests.gpu_support import (ATTN_MAX_ABS, ATTN_MEAN_ABS, assert_schedule_equal)
+
+    cfg = QWEN3_4B.with_(R=10, kv_dist=("uniform", 40, 700), V=512, layers=3)
+    inp, pipe = _state(cfg, 11, 3)
+    layers = 3
+    scale = 1.0 / math.sqrt(cfg.D)
+    t_ms = host(inp.t_ms)
+    table = host(inp.block_table)
+    kv_len = host(pipe.kv_len).astype(np.int64)
+    caches = host(pipe.kv_caches)                      # the oracle's own copy, float32 bits
+    flagged_total = 0
+    for rnd in range(5):
+        _refill(pipe, inp, cfg, rnd)
+        torch.cuda.synchronize()
+        ring = host(pipe.conf_ring)
+        q, kn, vn = host(pipe.q), host(pipe.k_new), host(pipe.v_new)
+        tl, dl = host(pipe.target_logits), host(pipe.draft_logits)
+        xt, ua, ur = host(pipe.draft_tokens), host(pipe.u_acc), host(pipe.u_res)
+
+        pipe.round(rnd)
+        torch.cuda.synchronize()
+
+        # schedule on the lagged confidence slot, with the lengths the chain has committed
+        conf = ring[oracle.lagged_round(rnd) % pipe.ring_depth]
+        sref = oracle.schedule_ref(conf, kv_len, t_ms, cfg.T_cap)
+        T = int(pipe.step.T.item())
+        sgpu = dict(verify_len=host(pipe.step.verify_len), q_offsets=host(pipe.step.q_offsets),
+                    markers=host(pipe.step.markers)[:T], T=T,
+                    objective=float(pipe.step.objective.item()))
+        assert assert_schedule_equal(sgpu, sref) == 0, f"round {rnd}: schedule flagged"
+        L, qo, mk = sref["verify_len"], sref["q_offsets"], sref["markers"]
+
+        # attention of every layer over the oracle's cache
+        for layer in range(layers):
+            ref = oracle.attn_ref_flat(q[layer, :T], kn[layer, :T], vn[layer, :T], caches[layer],
+                                       table, kv_len, mk, qo, scale, cfg.page_size)
+            err = np.abs(host(pipe.attn_out[layer, :T]).astype(np.float64) - ref)
+            assert err.max() <= ATTN_MAX_ABS and err.mean() <= ATTN_MEAN_ABS, \
+                (rnd, layer, err.max(), err.mean())
+
+        # acceptance, exact modulo flags
+        aref = oracle.accept_ref(tl[:T], dl, xt, L, qo, ua, ur, cfg.temperature)
+        agpu = dict(accepted_len=host(pipe.step.accepted_len),
+                    out_tokens=host(pipe.step.out_tokens), n_out=host(pipe.step.n_out))
+        nflag, _ = assert_accept_equal(agpu, aref)
+        flagged_total += nflag
+        accepted = np.where(aref["flagged"], agpu["accepted_len"], aref["accepted_len"])
+
+        # commit into the oracle's cache; the GPU's caches and lengths must match byte for byte
+        caches, kv_out, skipped = oracle.kv_commit_ref(kn, vn, caches, table, kv_len, qo,
+                                                       accepted, cfg.K, cfg.T_cap)
+        assert skipped == []
+        assert np.array_equal(host(pipe.kv_len), kv_out), rnd
+        assert np.array_equal(host(pipe.kv_caches), caches), rnd
+        assert np.all(kv_out == kv_len + accepted + 1)
+        kv_len = kv_out.astype(np.int64)
+    print(f"five chained rounds match the oracle chain; flagged requests: {flagged_total}")
+    assert binding().dspark_read_error() == 0

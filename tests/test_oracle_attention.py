@@ -135,3 +135,36 @@ def test_row_subset_matches_full():
     sub = _flat(c, 0.3, rows)
     for t, h in rows:
         assert np.array_equal(sub[t, h], full[t, h])
+
+
+def test_structured_keys_select_and_average_exactly():
+    """The closed form the full-size GPU checks use (tests/structured_attn.py): with keys that
+    select cache slots by a pseudo-random bit and coded values, each query's output is the mean
+    of the selected values and of its request's verify tokens up to itself.  The oracle must
+    reproduce it on a workload shaped like the large ones (page 64, D 128, GQA 4, several pages
+    per request, an empty cache, ragged last pages); the other keys weigh 2^-40 each."""
+    import math
+
+    from tests.structured_attn import install_structured, structured_expected
+    from workloads.configs import QWEN3_4B
+    from workloads.generate import build_step_inputs
+
+    cfg = QWEN3_4B.with_(R=4, Hq=8, Hkv=2, kv_dist=("uniform", 0, 300), V=16, layers=1)
+    inp = build_step_inputs(cfg, "cpu", seed=2, layers=1)
+    inp.kv_len[0] = 0                                  # an empty cache: only the verify tokens
+    install_structured(inp)
+    kv = inp.kv_len.numpy().astype(np.int64)
+    qo, mk = flatten_ref([5, 0, 3, 2], kv)
+    T = int(qo[-1])
+    f = lambda t: t.float().numpy().astype(np.float64)
+    got = attn_ref_flat(f(inp.q[0, :T]), f(inp.k_new[0, :T]), f(inp.v_new[0, :T]),
+                        f(inp.kv_caches[0]), inp.block_table.numpy(), kv, mk, qo,
+                        1.0 / math.sqrt(cfg.D), cfg.page_size)
+    ref = structured_expected(inp, qo, kv)             # [T][Hkv][D]
+    want = np.repeat(ref, cfg.G, axis=1)               # query head h reads KV head h // G
+    assert np.allclose(got, want, rtol=1e-9, atol=1e-9), np.abs(got - want).max()
+    # the selection matters: the plain mean over every visible key (scale 0) is far from it
+    uniform = attn_ref_flat(f(inp.q[0, :T]), f(inp.k_new[0, :T]), f(inp.v_new[0, :T]),
+                            f(inp.kv_caches[0]), inp.block_table.numpy(), kv, mk, qo, 0.0,
+                            cfg.page_size)
+    assert np.abs(uniform - want).max() > 0.1
