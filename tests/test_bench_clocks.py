@@ -27,7 +27,7 @@ def test_summary_parses_nvidia_smi_lines():
              "garbage line", ""]
     s = _sampler(lines)
     assert s == {"sm_mhz": 1785.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
-                 "samples": 3}
+                 "samples": 3, "sufficient": False}
     assert _sampler([]) is None
     s = _sampler(["1500, 1965, 700, 0x8, Not Active, Active, Not Active, Not Active"])
     assert s["reasons"] == ["hw_thermal_slowdown"]

@@ -103,11 +103,15 @@ def sweep_config(R: int) -> StepConfig:
         t_base_ms=5.0, t_slope_ms=0.004, t_knee=256)
 
 
+# the same workload verified greedily (the workload statement asks for greedy and T=0.7 runs)
+LONG_1024_GREEDY = LONG_1024.with_(name="lognormal-1024req-greedy", temperature=0.0)
+
 CONFIGS = {
     "tiny": TINY,
     "qwen3-4b-64req": QWEN3_4B,
     "mixed-256req": MIXED_256,
     "lognormal-1024req": LONG_1024,
+    "lognormal-1024req-greedy": LONG_1024_GREEDY,
 }
 for _R in SWEEP_LEVELS:
     CONFIGS[f"sweep-{_R}req"] = sweep_config(_R)
