@@ -122,12 +122,30 @@ int dspark_version(void);
  * verify_len  out int32 [R]; q_offsets out int32 [R + 1]; markers out int32 [T_cap][2]
  *             (entries past *T_out untouched); T_out out int32 [1]; objective out
  *             float64 [1] = f(n*).
+ * kv_len and markers may both be NULL: the call then decides the lengths and offsets only,
+ * which need nothing but the lagged confidences, so that a pipeline can schedule round i + 1
+ * while round i still runs; dspark_flatten_markers writes the markers once round i has
+ * committed the cache lengths.
  * Limits: 1 <= K <= DSPARK_MAX_K, R*K <= DSPARK_MAX_CANDIDATES.
  */
 int dspark_schedule(const float *conf_ring, int ring_depth, int round_idx, int R, int K,
                     const int32_t *kv_len, const double *t_ms, int T_cap,
                     int32_t *verify_len, int32_t *q_offsets, int32_t *markers,
                     int32_t *T_out, double *objective, dspark_stream_t stream);
+
+/*
+ * dspark_flatten_markers — the flattening step of dspark_schedule on its own.
+ *
+ * Defined by [P1 engineering table, row "内核利用率暴跌"] (verify tokens flattened, a marker
+ * tensor carries sequence membership and position) and row "GPU流水线停滞" (the scheduler
+ * runs ahead of the round it feeds).  markers[q_offsets[r] + j] = (r, kv_len[r] + j) for
+ * j = 0 .. q_offsets[r+1] - q_offsets[r] - 1, from the offsets of an earlier lengths-only
+ * dspark_schedule and the cache lengths current now.  kv_len int32 [R], q_offsets int32
+ * [R + 1], markers int32 [T_cap][2] (device).  A request whose offsets are not a flattening of
+ * 1..K+1 tokens inside [0, T_cap) sets DSPARK_DERR_OFFSETS and gets no markers.
+ */
+int dspark_flatten_markers(const int32_t *kv_len, const int32_t *q_offsets, int R, int K,
+                           int T_cap, int32_t *markers, dspark_stream_t stream);
 
 /*
  * Workspace of the attention pair (plan + calls).  rows = (Hq / Hkv) * (K + 1) query rows
@@ -142,8 +160,12 @@ size_t dspark_verify_attn_workspace_bytes(int R, int Hq, int Hkv, int D, int K);
  *
  * Work is the sequence of (request r, KV head g, unit) in request-major order, each request
  * contributing Hkv * (ceil(kv_len[r] / 64) + 8) units (its 64-key cache tiles, then eight
- * units standing for its own verify tokens and the segment's epilogue, which cost about as much
- * as eight cache tiles); the plan splits it into equal contiguous ranges, one per persistent CTA.
+ * units standing for its own verify tokens and the segment's epilogue).  The plan splits it
+ * into contiguous ranges, one per persistent CTA of the tensor-core kernel, chosen to minimise
+ * the largest modelled cost of a range: one per 64-key page, two for a segment's verify
+ * tokens, 3.5 per piece (a segment cut by range boundaries is computed in pieces) and 5.25 for
+ * merging a cut segment's partials; boundaries fall on even page counts and never inside a
+ * segment's verify-token units.  It runs a greedy fill for 1024 candidate bounds at once.
  * It also records, per request, the flattened offset, the token count and whether the
  * flattening is well formed (1 <= Q_r <= K + 1 tokens inside [0, T_cap), token j carrying the
  * marker (r, kv_len[r] + j)); a malformed request sets DSPARK_DERR_OFFSETS / _MARKER here and

@@ -84,6 +84,32 @@ struct ExpScale {
   }
 };
 
+// Eight consecutive logits as raw bits (one 16-byte load for bf16, two for f32), so that a
+// step's loads are all issued before any of them is converted.
+template <typename T> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> { uint4 a; };
+template <> struct Raw8<float> { float4 a, b; };
+__device__ __forceinline__ void load_raw8(const __nv_bfloat16 *p, Raw8<__nv_bfloat16> &r) {
+  r.a = __ldg(reinterpret_cast<const uint4 *>(p));
+}
+__device__ __forceinline__ void load_raw8(const float *p, Raw8<float> &r) {
+  r.a = __ldg(reinterpret_cast<const float4 *>(p));
+  r.b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+}
+__device__ __forceinline__ void cvt8(const Raw8<__nv_bfloat16> &r, float (&v)[8]) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&r.a);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void cvt8(const Raw8<float> &r, float (&v)[8]) {
+  v[0] = r.a.x; v[1] = r.a.y; v[2] = r.a.z; v[3] = r.a.w;
+  v[4] = r.b.x; v[5] = r.b.y; v[6] = r.b.z; v[7] = r.b.w;
+}
+
 // One CTA per scheduled logit row: one streaming pass with 16-byte loads, 32 elements per thread
 // and step; the running maximum rescales the float64 sum only when it rises.  GREEDY rows only
 // need the maximum and its lowest index.  Five CTAs per SM (registers capped to fit), so that a
@@ -112,17 +138,18 @@ accept_stats_kernel(const T *__restrict__ target, const T *__restrict__ draft, i
   double Z = 0.0;
   int amax = 0x7fffffff;
   // x[u][e] is element base[u] + e; groups are visited in index order
-  auto consume = [&](const float (&x)[4][8], const int (&base)[4]) {
+  auto consume = [&](const auto &x, const auto &base) {
+    constexpr int NU = sizeof(base) / sizeof(base[0]);
     if (GREEDY) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < NU; ++u)
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           if (x[u][e] > m) { m = x[u][e]; amax = base[u] + e; }
     } else {
       float lm = -INFINITY;
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < NU; ++u)
 #pragma unroll
         for (int e = 0; e < 8; ++e) lm = fmaxf(lm, x[u][e]);
       if (lm > m) {
@@ -132,7 +159,7 @@ accept_stats_kernel(const T *__restrict__ target, const T *__restrict__ draft, i
       if (m != -INFINITY) {
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < NU; ++u)
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
             s0 += exp2_sfu(c.mul(x[u][e] - m));
@@ -145,22 +172,38 @@ accept_stats_kernel(const T *__restrict__ target, const T *__restrict__ draft, i
   const bool vec = ((reinterpret_cast<uintptr_t>(row) & 15) == 0) && (V % 8 == 0) &&
                    (sizeof(T) == 2 || (reinterpret_cast<uintptr_t>(row) & 31) == 0);
   if (vec) {
+    // the next step's loads are issued before this step's values are used, so every thread
+    // keeps loads in flight while it computes
+    constexpr int kU = 2;
     const int nv = V / 8;
-    for (int v8 = tid; v8 < nv; v8 += 4 * kAccThreads) {
-      float x[4][8];
-      int base[4];
+    constexpr int kStep = kU * kAccThreads;
+    Raw8<T> cur[kU], nxt[kU];
+    auto issue = [&](Raw8<T>(&r)[kU], int v8) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kU; ++u) {
+        const int g = v8 + u * kAccThreads;
+        load_raw8(row + (size_t)(g < nv ? g : 0) * 8, r[u]);  // in bounds; masked below
+      }
+    };
+    if (tid < nv) issue(cur, tid);
+    for (int v8 = tid; v8 < nv; v8 += kStep) {
+      if (v8 + kStep < nv) issue(nxt, v8 + kStep);
+      float x[kU][8];
+      int base[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
         const int g = v8 + u * kAccThreads;
         base[u] = g * 8;
         if (g < nv) {
-          load8(row + (size_t)g * 8, x[u]);
+          cvt8(cur[u], x[u]);
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[u][e] = -INFINITY;
         }
       }
       consume(x, base);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) cur[u] = nxt[u];
     }
   } else {
     for (int b0 = tid * 8; b0 < V; b0 += 4 * kAccThreads * 8) {
@@ -229,32 +272,6 @@ struct RowPair {
     return fmaxf(0.f, pt - __fmul_rn(exp2_sfu(c.mul(zd - md)), invZd));
   }
 };
-
-// Eight consecutive logits as raw bits (one 16-byte load for bf16, two for f32), so that a
-// step's loads are all issued before any of them is converted.
-template <typename T> struct Raw8;
-template <> struct Raw8<__nv_bfloat16> { uint4 a; };
-template <> struct Raw8<float> { float4 a, b; };
-__device__ __forceinline__ void load_raw8(const __nv_bfloat16 *p, Raw8<__nv_bfloat16> &r) {
-  r.a = __ldg(reinterpret_cast<const uint4 *>(p));
-}
-__device__ __forceinline__ void load_raw8(const float *p, Raw8<float> &r) {
-  r.a = __ldg(reinterpret_cast<const float4 *>(p));
-  r.b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
-}
-__device__ __forceinline__ void cvt8(const Raw8<__nv_bfloat16> &r, float (&v)[8]) {
-  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&r.a);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __bfloat1622float2(h[i]);
-    v[2 * i] = f.x;
-    v[2 * i + 1] = f.y;
-  }
-}
-__device__ __forceinline__ void cvt8(const Raw8<float> &r, float (&v)[8]) {
-  v[0] = r.a.x; v[1] = r.a.y; v[2] = r.a.z; v[3] = r.a.w;
-  v[4] = r.b.x; v[5] = r.b.y; v[6] = r.b.z; v[7] = r.b.w;
-}
 
 // Logits [base, base + 8) of the row pair, element by element (any alignment; -inf past V).
 template <typename T>

@@ -8,11 +8,13 @@
 // (r, g); all G*Q_r query rows of the segment are processed together, so every KV byte is read
 // once.
 //
-// The unit sequence is split into equal contiguous ranges, one per persistent CTA (W units
-// each).  A segment cut by a range boundary is computed in pieces; each piece writes an
-// un-normalised (m, l, acc) partial and the last piece to arrive (atomic counter, no waiting)
-// merges them.  CTA c writes at most two partials: slot 2c for its first segment, 2c+1 for its
-// last one.
+// The unit sequence is split into contiguous ranges, one per persistent CTA.  A segment cut by a
+// range boundary is computed in pieces; each piece writes an un-normalised (m, l, acc) partial
+// and the last piece to arrive (atomic counter, no waiting) merges them.  CTA c writes at most
+// two partials: slot 2c for its first segment, 2c+1 for its last one.  The tensor-core kernel's
+// ranges come from the plan, which chooses them to minimise the largest modelled cost of a CTA
+// (cache pages, the verify-token tile, a fixed cost per piece and per merge); the CUDA-core
+// kernel splits the units into equal ranges.
 #pragma once
 
 #include "common.cuh"
@@ -25,8 +27,20 @@ constexpr int kMaxCtasPerSm = 4;
 struct AttnPlanHeader {
   int R, Hkv, rows_max, D;
   int tile_keys, total;  // total = units of the whole batch
-  int tc_ctas, tc_W;     // the tensor-core kernel's grid and units per CTA
+  int tc_ctas;           // the tensor-core kernel's grid (ranges in AttnWs::cta_begin)
+  float tc_bound;        // the largest modelled CTA cost of those ranges
 };
+
+// Cost model of the tensor-core kernel's work, in units of one 64-key cache page (fitted to a
+// per-CTA trace: 1.37 us per 128-key tile, 2.4 us per piece, 3.6 us per merge of split
+// partials).  A segment's verify tokens are one tile, its epilogue and the pipeline refill of
+// the next piece a piece cost; the head piece of a split segment usually merges, as the next
+// CTA finishes the segment's rest first.
+constexpr float kCostNewTile = 2.0f;
+constexpr float kCostPiece = 3.5f;
+constexpr float kCostMerge = 5.25f;
+// Candidate cost bounds the plan tests at once (one per thread of its single CTA).
+constexpr int kPlanThreads = 1024;
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -39,6 +53,7 @@ struct AttnWs {
   int *counters;     // [R * Hkv] arrival counters of split segments (kept at zero between calls)
   int4 *req;         // [R]: per request {t0, Q, kv_len, schedule valid} written by the plan
   int4 *cta_start;   // [max_ctas]: first segment of tensor-core CTA c {r, g, s0, units}, r < 0: none
+  int *cta_begin;    // [max_ctas + 1]: first unit of tensor-core CTA c; [tc_ctas] = total
   float *partials;   // [2 * max_ctas][rows_max][part_stride(D)]: acc[D], m, l per row
 };
 
@@ -50,6 +65,7 @@ __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, i
   const size_t o_cnt = off;                off += align256((size_t)R * Hkv * sizeof(int));
   const size_t o_req = off;                off += align256((size_t)R * sizeof(int4));
   const size_t o_cst = off;                off += align256((size_t)max_ctas * sizeof(int4));
+  const size_t o_beg = off;                off += align256((size_t)(max_ctas + 1) * sizeof(int));
   const size_t o_par = off;
   off += align256((size_t)2 * max_ctas * rows_max * part_stride(D) * sizeof(float));
   if (ws) {
@@ -59,6 +75,7 @@ __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, i
     ws->counters = reinterpret_cast<int *>(b + o_cnt);
     ws->req = reinterpret_cast<int4 *>(b + o_req);
     ws->cta_start = reinterpret_cast<int4 *>(b + o_cst);
+    ws->cta_begin = reinterpret_cast<int *>(b + o_beg);
     ws->partials = reinterpret_cast<float *>(b + o_par);
   }
   return off;
@@ -86,8 +103,45 @@ __host__ __device__ inline int segment_cache_tiles(int units) { return units - k
 __device__ __forceinline__ void find_segment(const int *__restrict__ tile_prefix, int R, int Hkv,
                                              int u, int &r, int &g, int &tiles, int &seg_start);
 
+// Greedy fill of CTAs in unit order under a cost bound: a segment goes whole into the current
+// CTA if it fits; otherwise the CTA takes a head piece of an even number of cache pages (at
+// least 2, with the piece and merge costs) and the rest continues in the next CTAs (which may
+// cut it again).  A range boundary never falls inside a segment's verify-token units.  Returns
+// the number of CTAs used (stops counting past `cap`); when `begin` is given, records the first
+// unit of every CTA used (begin[0] = 0).
+__device__ int plan_fill(const int *__restrict__ tile_prefix, int R, int Hkv, float bound,
+                         int cap, int *begin) {
+  int used = 1;
+  float cur = 0.f;
+  if (begin) begin[0] = 0;
+  for (int r = 0; r < R && used <= cap; ++r) {
+    const int seg_units = (tile_prefix[r + 1] - tile_prefix[r]) / Hkv;
+    const int u = seg_units - kSegTail;
+    for (int g = 0; g < Hkv && used <= cap; ++g) {
+      const int s0 = tile_prefix[r] + g * seg_units;
+      const float full = (float)u + kCostNewTile + kCostPiece;
+      if (cur + full <= bound) { cur += full; continue; }
+      int done = 0;  // cache pages of this segment placed in earlier CTAs
+      int head = (int)floorf(bound - cur - kCostPiece - kCostMerge);
+      head &= ~1;
+      if (head >= 2 && head < u) done = head;  // head piece in the current CTA
+      // the rest starts a new CTA; middle pieces fill whole CTAs while it does not fit
+      while (true) {
+        ++used;
+        if (begin && used <= cap) begin[used - 1] = s0 + done;
+        const float rest = (float)(u - done) + kCostNewTile + kCostPiece;
+        if (rest <= bound || used > cap) { cur = rest; break; }
+        int mid = (int)floorf(bound - kCostPiece) & ~1;
+        mid = max(mid, 2);
+        done = min(u, done + mid);
+      }
+    }
+  }
+  return used;
+}
+
 // It also records where each of the tensor-core kernel's `tc_ctas` CTAs starts (its first
-// segment), so that kernel walks segments in order without searching.
+// unit and first segment), so that kernel walks segments in order without searching.
 __global__ void __launch_bounds__(1024)
 attn_plan_kernel(const int32_t *__restrict__ kv_len, const int32_t *__restrict__ q_offsets,
                  const int32_t *__restrict__ markers, int R, int T_cap, int K, int Hkv,
@@ -147,12 +201,51 @@ attn_plan_kernel(const int32_t *__restrict__ kv_len, const int32_t *__restrict__
   }
   __syncthreads();  // tile_prefix complete (global writes of this block)
   const int total = ws.tile_prefix[R];
-  const int W = (total + tc_ctas - 1) / tc_ctas;
+
+  // Cost-balanced ranges: every thread runs the greedy fill below for one candidate bound on a
+  // CTA's modelled cost; the smallest bound that needs at most tc_ctas CTAs wins and its fill
+  // is run once more to record where each CTA starts.
+  __shared__ float s_tot;
+  __shared__ int s_best;
+  float seg_max = 0.f, mine = 0.f;
+  for (int r = tid; r < R; r += blockDim.x) {
+    const float u = (float)((ws.tile_prefix[r + 1] - ws.tile_prefix[r]) / Hkv - kSegTail);
+    const float full = u + kCostNewTile + kCostPiece;
+    mine += Hkv * full;
+    seg_max = fmaxf(seg_max, full);
+  }
+  mine = warp_sum(mine);
+  seg_max = warp_max(seg_max);
+  __shared__ float s_part[32], s_pmax[32];
+  if (lane == 0) { s_part[warp] = mine; s_pmax[warp] = seg_max; }
+  if (tid == 0) s_best = kPlanThreads;
+  __syncthreads();
+  if (tid == 0) {
+    float t = 0.f, mx = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) { t += s_part[w]; mx = fmaxf(mx, s_pmax[w]); }
+    s_tot = t;
+    s_pmax[0] = mx;
+  }
+  __syncthreads();
+  const float lo = s_tot / (float)tc_ctas;
+  const float hi = lo + s_pmax[0] + kCostMerge + kCostPiece;
+  const float bound = lo + (hi - lo) * (float)(tid + 1) / (float)blockDim.x;
+  if (plan_fill(ws.tile_prefix, R, Hkv, bound, tc_ctas, nullptr) <= tc_ctas) atomicMin(&s_best, tid);
+  __syncthreads();
+  const int best = min(s_best, (int)blockDim.x - 1);
+  if (tid == best) {
+    const int used = plan_fill(ws.tile_prefix, R, Hkv, bound, tc_ctas, ws.cta_begin);
+    // trailing CTAs get empty ranges; had no bound fitted, the last CTA would take the rest
+    for (int c = min(used, tc_ctas); c <= tc_ctas; ++c) ws.cta_begin[c] = total;
+    ws.hdr->tc_bound = bound;
+  }
+  __syncthreads();
   for (int c = tid; c < tc_ctas; c += blockDim.x) {
     int4 st = make_int4(-1, 0, 0, 0);
-    if (c * W < total) {
+    const int u0 = ws.cta_begin[c];
+    if (u0 < ws.cta_begin[c + 1]) {
       int r, g, tiles, s0;
-      find_segment(ws.tile_prefix, R, Hkv, c * W, r, g, tiles, s0);
+      find_segment(ws.tile_prefix, R, Hkv, u0, r, g, tiles, s0);
       st = make_int4(r, g, s0, tiles);
     }
     ws.cta_start[c] = st;
@@ -165,7 +258,6 @@ attn_plan_kernel(const int32_t *__restrict__ kv_len, const int32_t *__restrict__
     ws.hdr->tile_keys = kTileKeys;
     ws.hdr->total = total;
     ws.hdr->tc_ctas = tc_ctas;
-    ws.hdr->tc_W = W;
   }
 }
 
@@ -199,5 +291,30 @@ __device__ __forceinline__ int partial_slot(int c, int s0, int W) {
   const int first_cta = s0 / W;
   return 2 * c + ((c == first_cta && s0 != c * W) ? 1 : 0);
 }
+
+// The tensor-core kernel's CTA ranges: the plan's (begin[c] .. begin[c + 1]) when the grid is
+// the one the plan prepared, else equal ranges of W units.
+struct Ranges {
+  const int *begin;  // nullptr: equal ranges
+  int W, ctas, total;
+  __device__ __forceinline__ int start(int c) const {
+    return begin ? __ldcg(begin + c) : min(c * W, total);
+  }
+  // The CTA whose range holds unit u: the last c with start(c) <= u (empty ranges end the list).
+  __device__ __forceinline__ int cta_of(int u) const {
+    if (!begin) return u / W;
+    int lo = 0, hi = ctas - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldcg(begin + mid) <= u) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  }
+  // Slot of the partial CTA c writes for the segment starting at unit s0: 2c for the CTA's
+  // first segment, 2c + 1 for a segment that starts inside its range and continues past it.
+  __device__ __forceinline__ int slot(int c, int s0) const {
+    return 2 * c + ((c == cta_of(s0) && s0 != start(c)) ? 1 : 0);
+  }
+};
 
 }  // namespace dspark

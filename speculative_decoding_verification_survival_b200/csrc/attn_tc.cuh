@@ -76,7 +76,8 @@ constexpr int kPS = part_stride(kD);                 // floats per split-KV part
 constexpr uint32_t kBarKFull = 0, kBarVFull = 64, kBarKEmpty = 128, kBarVEmpty = 192,
                    kBarSFull = 256, kBarPFull = 272, kBarODone = 280, kBarQFull = 288,
                    kBarQEmpty = 296, kBarOFree = 304, kBarDrain = 312;
-constexpr uint32_t kAuxTmem = 320, kAuxAbort = 324, kAuxLast = 328, kAuxPmax = 512,
+constexpr uint32_t kAuxTmem = 320, kAuxAbort = 324, kAuxLast = 328, kAuxSplit = 336,
+                   kAuxPmax = 512,
                    kAuxLsum = 512 + 2 * kSoftmaxThreads * 4;
 
 constexpr uint32_t kTmemCols = 512;
@@ -121,23 +122,30 @@ __device__ __forceinline__ Meta piece_meta(const AttnArgs &a, int r, int ta, int
 // This CTA's contiguous range of units [u, u1) as pieces (one per segment it touches), walking
 // the segments in order from the CTA's start record written by the plan.
 struct PieceIter {
-  int u, u1, W;
+  int u, u1;
+  Ranges rg;
   int r, g, tiles, s0;  // current segment
   __device__ __forceinline__ void init(const AttnArgs &a) {
     const int total = __ldg(&a.ws.hdr->total);
     const int ctas = __ldg(&a.ws.hdr->tc_ctas);
-    if (ctas == (int)gridDim.x) {
-      W = __ldg(&a.ws.hdr->tc_W);
+    if (ctas == (int)gridDim.x) {  // the plan's cost-balanced ranges
+      rg.begin = a.ws.cta_begin;
+      rg.W = 0;
+      rg.ctas = ctas;
+      rg.total = total;
       const int4 st = __ldg(a.ws.cta_start + blockIdx.x);
       r = st.x; g = st.y; s0 = st.z; tiles = st.w;
-    } else {  // a grid the plan did not prepare for: search for the first segment
-      W = (total + gridDim.x - 1) / gridDim.x;
+    } else {  // a grid the plan did not prepare for: equal ranges, search the first segment
+      rg.begin = nullptr;
+      rg.W = (total + gridDim.x - 1) / gridDim.x;
+      rg.ctas = gridDim.x;
+      rg.total = total;
       r = -1;
-      if ((int64_t)blockIdx.x * W < total)
-        find_segment(a.ws.tile_prefix, a.R, a.Hkv, blockIdx.x * W, r, g, tiles, s0);
+      if ((int64_t)blockIdx.x * rg.W < total)
+        find_segment(a.ws.tile_prefix, a.R, a.Hkv, blockIdx.x * rg.W, r, g, tiles, s0);
     }
-    u = blockIdx.x * W;
-    u1 = (r < 0) ? u : min(u + W, total);
+    u = rg.start(blockIdx.x);
+    u1 = (r < 0) ? u : min(rg.start(blockIdx.x + 1), total);
   }
   __device__ __forceinline__ bool next(const AttnArgs &a, int &r_, int &g_, int &ta, int &tb,
                                        int &tiles_, int &s0_) {
@@ -312,6 +320,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
   float *lsum_buf = reinterpret_cast<float *>(gaux + kAuxLsum);
   const uint32_t stage = base + kOffStage;
   volatile int *s_last = reinterpret_cast<volatile int *>(gaux + kAuxLast);
+  volatile int *s_split = reinterpret_cast<volatile int *>(gaux + kAuxSplit);  // [3]
   // ring r (0 = K d-half 0, 1 = K d-half 1, 2 = V d-half 0, 3 = V d-half 1), page slot s
   auto ring = [&](int rg, uint32_t s) {
     return base + (rg < 2 ? (uint32_t)rg * kRingBytesK
@@ -583,7 +592,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       // its own partial; this early read keeps the counter's latency off the epilogue.
       const bool split = !(ta == 0 && tb == tiles);
       int pre_count = -1;
-      if (tid == 0 && split) pre_count = ptx::ld_acquire_gpu(a.ws.counters + r * a.Hkv + g);
+      if (tid == 0 && split) {
+        pre_count = ptx::ld_acquire_gpu(a.ws.counters + r * a.Hkv + g);
+        // the CTAs holding this segment's pieces and the slot of its first piece's partial
+        // (read by everyone after the epilogue's first barrier)
+        const int c_first = ta == 0 ? (int)blockIdx.x : it.rg.cta_of(s0);
+        const int c_last = tb == tiles ? (int)blockIdx.x : it.rg.cta_of(s0 + tiles - 1);
+        s_split[0] = c_first;
+        s_split[1] = c_last;
+        s_split[2] = 2 * c_first + (s0 != it.rg.start(c_first) ? 1 : 0);
+      }
       SoftmaxState sm;
       sm.m_run = -INFINITY;
       sm.l_part = 0.f;
@@ -655,13 +673,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
         ptx::tc_fence_after();
       }
       if (tid == 0 && split) {  // 2: merge at once (read after the next barrier)
-        const int pieces = (s0 + tiles - 1) / it.W - s0 / it.W + 1;
+        const int pieces = s_split[1] - s_split[0] + 1;
         *s_last = (pre_count == pieces - 1) ? 2 : 0;
       }
       ptx::named_bar_sync(2, kSoftmaxThreads);
       const bool whole = (ta == 0 && tb == tiles);
-      const int W = it.W;
-      float *part = a.ws.partials + (size_t)partial_slot(blockIdx.x, s0, W) * a.rows_max * kPS;
+      const int c_first = s_split[0], c_last = s_split[1], slot_first = s_split[2];
+      const int my_slot = ((int)blockIdx.x == c_first) ? slot_first : 2 * (int)blockIdx.x;
+      float *part = a.ws.partials + (size_t)my_slot * a.rows_max * kPS;
       if (m.ntiles > 0) {
         float l = 0.f;
         for (int cc = 0; cc < m.C; ++cc) l += lsum_buf[rho + cc * rpc] + lsum_buf[128 + rho + cc * rpc];
@@ -740,7 +759,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
           __threadfence();
           ptx::named_bar_sync(2, kSoftmaxThreads);
           if (tid == 0) {
-            const int pieces = (s0 + tiles - 1) / W - s0 / W + 1;
+            const int pieces = c_last - c_first + 1;
             const int prev = atomicAdd(a.ws.counters + r * a.Hkv + g, 1);
             *s_last = (prev == pieces - 1);
           }
@@ -752,7 +771,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
         ptx::named_bar_sync(2, kSoftmaxThreads);
         if (*s_last) {
           __threadfence();
-          const int c_first = s0 / W, c_last = (s0 + tiles - 1) / W;
           const size_t pstride = (size_t)a.rows_max * kPS;
           const float *P0 = a.ws.partials;
           // items (row, float4 column), four per thread: each item merges the pieces online,
@@ -773,7 +791,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
               float4 v[2][4];
 #pragma unroll
               for (int pc = 0; pc < 2; ++pc) {
-                const float *Pp = P0 + (size_t)partial_slot(min(c2 + pc, c_last), s0, W) * pstride;
+                const int cc = min(c2 + pc, c_last);
+                const float *Pp = P0 + (size_t)(cc == c_first ? slot_first : 2 * cc) * pstride;
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                   const int item = min(it0 + k * kSoftmaxThreads, nitems - 1);

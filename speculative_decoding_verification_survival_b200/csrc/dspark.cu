@@ -111,9 +111,9 @@ int dspark_schedule(const float *conf_ring, int ring_depth, int round_idx, int R
                     const int32_t *kv_len, const double *t_ms, int T_cap, int32_t *verify_len,
                     int32_t *q_offsets, int32_t *markers, int32_t *T_out, double *objective,
                     dspark_stream_t stream) {
-  if (!conf_ring || !kv_len || !t_ms || !verify_len || !q_offsets || !markers || !T_out ||
-      !objective)
+  if (!conf_ring || !t_ms || !verify_len || !q_offsets || !T_out || !objective)
     return DSPARK_EINVAL;
+  if ((kv_len == nullptr) != (markers == nullptr)) return DSPARK_EINVAL;  // both or neither
   if (R < 1 || K < 1 || K > DSPARK_MAX_K || ring_depth < DSPARK_CONF_LAG + 1 || round_idx < 0 ||
       T_cap < R)
     return DSPARK_EINVAL;
@@ -141,6 +141,15 @@ int dspark_schedule(const float *conf_ring, int ring_depth, int round_idx, int R
     default: return DSPARK_EUNSUPPORTED;
   }
 #undef DSPARK_SCHED_LAUNCH
+  return launch_status();
+}
+
+int dspark_flatten_markers(const int32_t *kv_len, const int32_t *q_offsets, int R, int K,
+                           int T_cap, int32_t *markers, dspark_stream_t stream) {
+  if (!kv_len || !q_offsets || !markers || R < 1 || K < 1 || K > DSPARK_MAX_K || T_cap < R)
+    return DSPARK_EINVAL;
+  flatten_markers_kernel<<<(R + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      kv_len, q_offsets, R, K, T_cap, markers);
   return launch_status();
 }
 

@@ -17,7 +17,9 @@
 //      Passes whose digit is the same for every key are skipped.
 //   3. Prefix sums of the sorted S (float64; sequential per thread, tree across threads),
 //      f(n) = (R + P(n)) / t_ms[R + n], n* = first n with f(n+1) <= f(n).
-//   4. verify_len by counting the first n* payloads, exclusive scan into q_offsets, markers.
+//   4. verify_len by counting the first n* payloads, exclusive scan into q_offsets, markers
+//      (or, for a lengths-only call, no markers: flatten_markers_kernel writes them later from
+//      the cache lengths current then).
 #pragma once
 
 #include "common.cuh"
@@ -271,13 +273,15 @@ schedule_kernel(const float *__restrict__ conf_ring, int ring_depth, int round_i
     const int r = tid * per + i;
     if (r < R) {
       const int L = Lcnt[r];
-      int n = kv_len[r];
-      if (n < 0) { raise_error(DSPARK_DERR_KV_LEN); n = 0; }
       verify_len[r] = L;
       q_offsets[r] = (int32_t)off;
-      for (int j = 0; j <= L; ++j) {
-        markers[2 * (off + j)] = r;
-        markers[2 * (off + j) + 1] = n + j;
+      if (markers != nullptr) {  // lengths-only calls leave the markers to flatten_markers_kernel
+        int n = kv_len[r];
+        if (n < 0) { raise_error(DSPARK_DERR_KV_LEN); n = 0; }
+        for (int j = 0; j <= L; ++j) {
+          markers[2 * (off + j)] = r;
+          markers[2 * (off + j) + 1] = n + j;
+        }
       }
       off += 1u + (uint32_t)L;
       if (r == R - 1) {
@@ -285,6 +289,28 @@ schedule_kernel(const float *__restrict__ conf_ring, int ring_depth, int round_i
         *T_out = (int32_t)off;
       }
     }
+  }
+}
+
+// The flattening step alone: markers[q_offsets[r] + j] = (r, kv_len[r] + j), j < Q_r, from
+// offsets a lengths-only schedule wrote earlier and the cache lengths current now.  One thread
+// per request; offsets that are not a valid flattening within T_cap raise DSPARK_DERR_OFFSETS
+// and that request's markers are not written.
+__global__ void flatten_markers_kernel(const int32_t *__restrict__ kv_len,
+                                       const int32_t *__restrict__ q_offsets, int R, int K,
+                                       int T_cap, int32_t *__restrict__ markers) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= R) return;
+  const int t0 = q_offsets[r], Q = q_offsets[r + 1] - t0;
+  if (Q < 1 || Q > K + 1 || t0 < 0 || t0 > T_cap - Q) {
+    raise_error(DSPARK_DERR_OFFSETS);
+    return;
+  }
+  int n = kv_len[r];
+  if (n < 0) { raise_error(DSPARK_DERR_KV_LEN); n = 0; }
+  for (int j = 0; j < Q; ++j) {
+    markers[2 * (t0 + j)] = r;
+    markers[2 * (t0 + j) + 1] = n + j;
   }
 }
 

@@ -53,6 +53,7 @@ _SIGS = {
     "dspark_status_string": ([_i], ctypes.c_char_p),
     "dspark_version": ([], _i),
     "dspark_schedule": ([_p, _i, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p], _i),
+    "dspark_flatten_markers": ([_p, _p, _i, _i, _i, _p, _p], _i),
     "dspark_verify_attn_workspace_bytes": ([_i, _i, _i, _i, _i], _sz),
     "dspark_verify_attn_plan": ([_p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _sz, _p], _i),
     "dspark_verify_attn": ([_p, _p, _p, _p, _i64, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i,
@@ -128,7 +129,7 @@ def dspark_schedule(conf_ring, round_idx, kv_len, t_ms, T_cap, verify_len, q_off
                     T_out, objective, stream=None):
     """conf_ring float32 [depth][R][K]; kv_len int32 [R]; t_ms float64 [T_cap+1];
     outputs verify_len int32 [R], q_offsets int32 [R+1], markers int32 [T_cap][2],
-    T_out int32 [1], objective float64 [1]."""
+    T_out int32 [1], objective float64 [1].  kv_len = markers = None: lengths only."""
     depth, R, K = conf_ring.shape
     _check(conf_ring, torch.float32, "conf_ring")
     _check(kv_len, torch.int32, "kv_len")
@@ -136,6 +137,15 @@ def dspark_schedule(conf_ring, round_idx, kv_len, t_ms, T_cap, verify_len, q_off
     _call("dspark_schedule", _ptr(conf_ring), depth, int(round_idx), R, K, _ptr(kv_len),
           _ptr(t_ms), int(T_cap), _ptr(verify_len), _ptr(q_offsets), _ptr(markers), _ptr(T_out),
           _ptr(objective), _stream(stream))
+
+
+def dspark_flatten_markers(kv_len, q_offsets, K, markers, stream=None):
+    """kv_len int32 [R]; q_offsets int32 [R+1] (from a lengths-only schedule); markers out
+    int32 [T_cap][2]."""
+    for t, n in ((kv_len, "kv_len"), (q_offsets, "q_offsets"), (markers, "markers")):
+        _check(t, torch.int32, n)
+    _call("dspark_flatten_markers", _ptr(kv_len), _ptr(q_offsets), kv_len.shape[0], int(K),
+          markers.shape[0], _ptr(markers), _stream(stream))
 
 
 def dspark_verify_attn_workspace_bytes(R, Hq, Hkv, D, K) -> int:

@@ -42,6 +42,17 @@ class VerifyStep:
         _d.dspark_schedule(conf_ring, round_idx, kv_len, t_ms, self.T_cap, self.verify_len,
                            self.q_offsets, self.markers, self.T, self.objective, stream)
 
+    def schedule_lengths(self, conf_ring, round_idx, t_ms, stream=None):
+        """The schedule's decision alone (verify lengths, offsets, T, objective): it reads only
+        the lagged confidences and the step-time table, so it may run before the previous
+        round has committed its cache lengths; flatten() then writes the markers."""
+        _d.dspark_schedule(conf_ring, round_idx, None, t_ms, self.T_cap, self.verify_len,
+                           self.q_offsets, None, self.T, self.objective, stream)
+
+    def flatten(self, kv_len, stream=None):
+        """Markers of the scheduled lengths at the current cache lengths."""
+        _d.dspark_flatten_markers(kv_len, self.q_offsets, self.K, self.markers, stream)
+
     def plan(self, kv_len, stream=None):
         _d.dspark_verify_attn_plan(kv_len, self.q_offsets, self.markers, self.R, self.Hq,
                                    self.Hkv, self.D, self.K, self.attn_ws, stream)

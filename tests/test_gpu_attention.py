@@ -236,3 +236,76 @@ def test_full_workload_structured_keys_and_values(name):
     assert not bad.any(), (f"{int(bad.sum())} of {bad.size} elements off, worst "
                            f"{float((err - bound).max()):.3e} at {np.argwhere(bad)[0].tolist()}")
     assert binding().dspark_read_error() == 0
+
+
+# ---- the plan's cost-balanced ranges ----------------------------------------------------------
+_COST_NEW, _COST_PIECE, _COST_MERGE, _SEG_TAIL = 2.0, 3.5, 5.25, 8
+
+
+def _plan_ranges(step, cfg):
+    """The tensor-core kernel's CTA ranges as the plan wrote them into the workspace (layout of
+    the workspace: header, unit prefix, counters, request records, CTA start records, CTA
+    range starts, each 256-byte aligned)."""
+    al = lambda x: (x + 255) // 256 * 256
+    ws = step.attn_ws.cpu().numpy()
+    hdr = ws[:32].view(np.int32)
+    total, ctas = int(hdr[5]), int(hdr[6])
+    bound = float(ws[28:32].view(np.float32)[0])
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    off = al(32)
+    prefix = ws[off:off + 4 * (cfg.R + 1)].view(np.int32).astype(np.int64)
+    off += al(4 * (cfg.R + 1)) + al(4 * cfg.R * cfg.Hkv) + al(16 * cfg.R) + al(16 * 4 * sms)
+    begin = ws[off:off + 4 * (ctas + 1)].view(np.int32).astype(np.int64)
+    return total, ctas, bound, prefix, begin
+
+
+def _range_costs(prefix, Hkv, begin):
+    """Modelled cost of every CTA's range (cache pages + verify tile + per piece + merge of a
+    split segment's head piece)."""
+    seg_units = np.diff(prefix) // Hkv
+    starts = np.concatenate([prefix[r] + g * seg_units[r] + np.zeros(1, np.int64)
+                             for r in range(len(seg_units)) for g in range(Hkv)])
+    lens = np.repeat(seg_units, Hkv)
+    costs = np.zeros(len(begin) - 1)
+    for c in range(len(begin) - 1):
+        u0, u1 = begin[c], begin[c + 1]
+        if u0 >= u1:
+            continue
+        for s0, n in zip(starts, lens):
+            a, b = max(u0, s0), min(u1, s0 + n)
+            if a >= b:
+                continue
+            cache = n - _SEG_TAIL
+            pages = min(b, s0 + cache) - min(a, s0 + cache)
+            cost = pages + _COST_PIECE + (_COST_NEW if b == s0 + n else 0.0)
+            if a == s0 and b < s0 + n:
+                cost += _COST_MERGE          # the head piece of a split segment merges
+            costs[c] += cost
+    return costs, starts, lens
+
+
+@pytest.mark.parametrize("name", ["qwen3-4b-64req", "sweep-1req", "sweep-128req"])
+def test_plan_ranges_are_cost_balanced(name):
+    cfg = CONFIGS[name]
+    inp = build_step_inputs(cfg, "cuda", seed=0, layers=1)
+    step = new_step(cfg)
+    step.schedule(inp.conf_ring, inp.round_idx, inp.kv_len, inp.t_ms)
+    step.plan(inp.kv_len)
+    torch.cuda.synchronize()
+    total, ctas, bound, prefix, begin = _plan_ranges(step, cfg)
+    assert begin[0] == 0 and begin[-1] == total and np.all(np.diff(begin) >= 0)
+    costs, starts, lens = _range_costs(prefix, cfg.Hkv, begin)
+    # no range boundary inside a segment's verify-token units
+    for b in begin[1:-1]:
+        k = np.searchsorted(starts, b, side="right") - 1
+        assert b - starts[k] <= lens[k] - _SEG_TAIL or b == starts[k] + lens[k]
+    assert costs.max() <= bound + 1e-3
+    # no worse than equal ranges under the same model, up to the spacing of the bounds the
+    # plan tries (1024 between the mean cost and the mean plus the largest segment's)
+    W = -(-total // ctas)
+    equal = np.minimum(np.arange(ctas + 1) * W, total)
+    eq_costs, _, _ = _range_costs(prefix, cfg.Hkv, equal)
+    spacing = ((lens - _SEG_TAIL).max() + _COST_NEW + 2 * _COST_PIECE + _COST_MERGE) / 1024
+    assert costs.max() <= eq_costs.max() + spacing, (costs.max(), eq_costs.max())
+    print(f"{name}: largest modelled CTA cost {costs.max():.1f} (equal ranges "
+          f"{eq_costs.max():.1f}), mean {costs.sum() / ctas:.1f}")

@@ -14,7 +14,7 @@ from workloads.generate import build_step_inputs, flatten_target
 pytestmark = pytest.mark.gpu
 
 
-def _state(cfg, seed, layers):
+def _state(cfg, seed, layers, overlap=False):
     from speculative_decoding_verification_survival_b200 import RoundPipeline
     inp = build_step_inputs(cfg, "cuda", seed=seed, layers=layers, kv_copies=1,
                             reserve_tokens=8 * (cfg.K + 1))
@@ -25,7 +25,8 @@ def _state(cfg, seed, layers):
     pipe = RoundPipeline(step, inp.conf_ring.clone(), inp.t_ms, inp.kv_len.clone(),
                          inp.block_table, inp.q.clone(), inp.k_new.clone(), inp.v_new.clone(),
                          caches, attn_out, tflat, inp.draft_logits.clone(), inp.draft_tokens.clone(),
-                         inp.u_acc.clone(), inp.u_res.clone(), cfg.temperature)
+                         inp.u_acc.clone(), inp.u_res.clone(), cfg.temperature,
+                         overlap=overlap)
     return inp, pipe
 
 
@@ -99,7 +100,8 @@ def test_captured_step_replays_the_eager_step():
         assert torch.equal(a, b)
 
 
-def test_graph_rounds_follow_the_oracle_chain():
+@pytest.mark.parametrize("overlap", [False, True])
+def test_graph_rounds_follow_the_oracle_chain(overlap):
     """Five rounds replayed as CUDA graphs, each checked against the oracle chain run on the
     same input bits: schedule_ref on the confidences of two rounds earlier, attn_ref_flat per
     layer over the oracle's own cache, accept_ref, kv_commit_ref, and the committed lengths
@@ -112,7 +114,7 @@ def test_graph_rounds_follow_the_oracle_chain():
     from tests.gpu_support import (ATTN_MAX_ABS, ATTN_MEAN_ABS, assert_schedule_equal)
 
     cfg = QWEN3_4B.with_(R=10, kv_dist=("uniform", 40, 700), V=512, layers=3)
-    inp, pipe = _state(cfg, 11, 3)
+    inp, pipe = _state(cfg, 11, 3, overlap=overlap)
     layers = 3
     scale = 1.0 / math.sqrt(cfg.D)
     t_ms = host(inp.t_ms)
@@ -130,14 +132,14 @@ def test_graph_rounds_follow_the_oracle_chain():
 
         pipe.round(rnd)
         torch.cuda.synchronize()
+        st = pipe.step_of(rnd)
 
         # schedule on the lagged confidence slot, with the lengths the chain has committed
         conf = ring[oracle.lagged_round(rnd) % pipe.ring_depth]
         sref = oracle.schedule_ref(conf, kv_len, t_ms, cfg.T_cap)
-        T = int(pipe.step.T.item())
-        sgpu = dict(verify_len=host(pipe.step.verify_len), q_offsets=host(pipe.step.q_offsets),
-                    markers=host(pipe.step.markers)[:T], T=T,
-                    objective=float(pipe.step.objective.item()))
+        T = int(st.T.item())
+        sgpu = dict(verify_len=host(st.verify_len), q_offsets=host(st.q_offsets),
+                    markers=host(st.markers)[:T], T=T, objective=float(st.objective.item()))
         assert assert_schedule_equal(sgpu, sref) == 0, f"round {rnd}: schedule flagged"
         L, qo, mk = sref["verify_len"], sref["q_offsets"], sref["markers"]
 
@@ -151,8 +153,8 @@ def test_graph_rounds_follow_the_oracle_chain():
 
         # acceptance, exact modulo flags
         aref = oracle.accept_ref(tl[:T], dl, xt, L, qo, ua, ur, cfg.temperature)
-        agpu = dict(accepted_len=host(pipe.step.accepted_len),
-                    out_tokens=host(pipe.step.out_tokens), n_out=host(pipe.step.n_out))
+        agpu = dict(accepted_len=host(st.accepted_len), out_tokens=host(st.out_tokens),
+                    n_out=host(st.n_out))
         nflag, _ = assert_accept_equal(agpu, aref)
         flagged_total += nflag
         accepted = np.where(aref["flagged"], agpu["accepted_len"], aref["accepted_len"])
@@ -166,4 +168,29 @@ def test_graph_rounds_follow_the_oracle_chain():
         assert np.all(kv_out == kv_len + accepted + 1)
         kv_len = kv_out.astype(np.int64)
     print(f"five chained rounds match the oracle chain; flagged requests: {flagged_total}")
+    assert binding().dspark_read_error() == 0
+
+
+def test_overlapped_rounds_equal_serial_rounds():
+    """Round i + 1's scheduling decision on a side stream, concurrent with round i, gives the
+    serial chain's results bit for bit, as graphs and eagerly."""
+    cfg = QWEN3_4B.with_(R=14, kv_dist=("uniform", 40, 900), V=256, layers=2)
+    inp_a, serial = _state(cfg, 5, 2)
+    inp_b, overlap = _state(cfg, 5, 2, overlap=True)
+    inp_c, eager = _state(cfg, 5, 2, overlap=True)
+    for rnd in range(6):
+        for p, i in ((serial, inp_a), (overlap, inp_b), (eager, inp_c)):
+            _refill(p, i, cfg, rnd)
+        serial.round(rnd)
+        overlap.round(rnd)
+        eager.round(rnd, graph=False)
+        torch.cuda.synchronize()
+        for other in (overlap, eager):
+            for name in ("kv_len", "attn_out", "kv_caches"):
+                assert torch.equal(getattr(serial, name), getattr(other, name)), (rnd, name)
+            for name in ("verify_len", "q_offsets", "accepted_len", "out_tokens", "n_out"):
+                assert torch.equal(getattr(serial.step, name),
+                                   getattr(other.step_of(rnd), name)), (rnd, name)
+            T = int(serial.step.T.item())
+            assert torch.equal(serial.step.markers[:T], other.step_of(rnd).markers[:T])
     assert binding().dspark_read_error() == 0
