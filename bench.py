@@ -767,6 +767,9 @@ def main():
     ap.add_argument("--impl", default="dspark", choices=["dspark", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(CONFIGS))
     ap.add_argument("--layers", type=int, default=36)
+    ap.add_argument("--requests", type=int, default=None,
+                    help="the workload with this many requests instead (a smaller case of the "
+                         "same distributions, e.g. for an ncu capture)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-parity", action="store_true")
     ap.add_argument("--report", action="store_true",
@@ -797,6 +800,8 @@ def main():
     rows = []
     for name in workloads:
         cfg = CONFIGS[name].with_(layers=args.layers)
+        if args.requests:
+            cfg = cfg.with_(R=args.requests, name=f"{cfg.name}@{args.requests}req")
         S, res = run_dspark(args, cfg, rank, world, device, with_e2e=not args.report)
         agg = reduce_replicas(res["ms_total"] / args.steps, res["attn_ms"],
                               res["e2e"]["ms"] if res["e2e"] else 0.0,

@@ -131,7 +131,8 @@ __device__ int plan_fill(const int *__restrict__ tile_prefix, int R, int Hkv, fl
         if (begin && used <= cap) begin[used - 1] = s0 + done;
         const float rest = (float)(u - done) + kCostNewTile + kCostPiece;
         if (rest <= bound || used > cap) { cur = rest; break; }
-        int mid = (int)floorf(bound - kCostPiece) & ~1;
+        // a segment cut from its start here (no head piece placed above) has its head now
+        int mid = (int)floorf(bound - kCostPiece - (done == 0 ? kCostMerge : 0.f)) & ~1;
         mid = max(mid, 2);
         done = min(u, done + mid);
       }

