@@ -424,6 +424,15 @@ def request_attn_inputs(S, r, qo, mk, layer=0):
                 kv_len=np.array([n]), markers=markers, q_offsets=np.array([0, t1 - t0]))
 
 
+def split_by_kv_head(d, G):
+    """The same request's attention as Hkv independent problems, one per KV head (its G query
+    heads, its K/V rows): exactly the same arithmetic, in pieces a process pool can balance."""
+    Hkv = d["k_new"].shape[1]
+    return [dict(d, q=d["q"][:, g * G:(g + 1) * G], k_new=d["k_new"][:, g:g + 1],
+                 v_new=d["v_new"][:, g:g + 1], kv_pages=d["kv_pages"][:, :, g:g + 1].copy())
+            for g in range(Hkv)]
+
+
 def _oracle_attn_task(args):
     """One request's attention in the oracle (every token, every query head); seconds taken."""
     from threadpoolctl import threadpool_limits
@@ -568,7 +577,8 @@ def cpu_baseline(S, pool, n_workers, single_thread=True):
         t_sched = time.perf_counter() - t0
     qo, mk = s["q_offsets"], s["markers"]
     scale = 1.0 / math.sqrt(cfg.D)
-    attn_tasks = [(request_attn_inputs(S, r, qo, mk), scale, cfg.page_size) for r in picked]
+    attn_tasks = [(part, scale, cfg.page_size) for r in picked
+                  for part in split_by_kv_head(request_attn_inputs(S, r, qo, mk), cfg.G)]
     acc_tasks = [accept_chunk_args(S, r0, min(n_acc, r0 + 4), qo) for r0 in range(0, n_acc, 4)]
 
     def scaled(t_attn, t_acc):
@@ -591,7 +601,8 @@ def cpu_baseline(S, pool, n_workers, single_thread=True):
     tokens = float(S.L.sum())
     blas = [dict(api=i.get("internal_api"), threads=i.get("num_threads")) for i in threadpool_info()]
     sample = (f"oracle (float64 NumPy), one layer call's attention of {len(picked)} whole requests "
-              f"(every token and head; {sample_units / all_units:.4f} of the call's work) scaled "
+              f"(every token and head, one task per KV head; {sample_units / all_units:.4f} of the "
+              f"call's work) scaled "
               f"to {cfg.R} requests x {cfg.layers} calls, acceptance of {n_acc} requests scaled "
               f"to {cfg.R}, schedule of all {cfg.R}; run on {n_workers} worker processes of one "
               f"thread each (single-thread figure beside it)")
