@@ -376,33 +376,57 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
   if (warp == kWarpK || warp == kWarpV) {
     // ------------------------------------------------------------------ TMA producers
     // one warp loads K, another V (a bulk L2 prefetch of later pages was tried and only
-    // lengthened the loads' latency).  Tile gt
-    // uses page slots 2(gt mod 3) and 2(gt mod 3) + 1 of both rings' families.
-    if (lane == 0) {
-      const bool is_k = (warp == kWarpK);
-      const uint32_t full0 = is_k ? kBarKFull : kBarVFull, empty0 = is_k ? kBarKEmpty : kBarVEmpty;
-      const int rg0 = is_k ? 0 : 2;
-      const CUtensorMap *nmap = is_k ? &tmap_kn : &tmap_vn;
-      const int nslots = is_k ? kSlotsK : kSlotsV;
-      // every cached page is read by exactly one CTA once: let it leave L2 first, so that the
-      // split-KV partials written early in the kernel are still there when they are merged
-      const uint64_t stream_policy = ptx::l2_policy_evict_first();
-      int last_use[kMaxSlots];  // latest slot use that was armed (TMA or empty arrive), -1 if none
+    // lengthened the loads' latency).  Tile gt uses page slots 2(gt mod 3) and 2(gt mod 3) + 1
+    // of both rings' families.  The whole warp walks the tiles; lane 0 waits on the barriers
+    // and issues the copies.  The block-table entries come 32 at a time, lane i holding entry
+    // base + i, and the chunk after the current one is loaded ahead: a page's lookup is a
+    // register shuffle, so no copy waits for a dependent global load (under the kernel's own
+    // traffic that load took about 1000 cycles and held back every page's copy).
+    const bool is_k = (warp == kWarpK);
+    const uint32_t full0 = is_k ? kBarKFull : kBarVFull, empty0 = is_k ? kBarKEmpty : kBarVEmpty;
+    const int rg0 = is_k ? 0 : 2;
+    const CUtensorMap *nmap = is_k ? &tmap_kn : &tmap_vn;
+    const int nslots = is_k ? kSlotsK : kSlotsV;
+    // every cached page is read by exactly one CTA once: let it leave L2 first, so that the
+    // split-KV partials written early in the kernel are still there when they are merged
+    const uint64_t stream_policy = ptx::l2_policy_evict_first();
+    int last_use[kMaxSlots];  // latest slot use that was armed (TMA or empty arrive), -1 if none
 #pragma unroll
-      for (int k = 0; k < kMaxSlots; ++k) last_use[k] = -1;
-      TileCursor tc;
-      tc.init(a);
-      while (tc.ok && !*abort_flag) {
-        const Meta &m = tc.m;
-        for (int h = 0; h < 2; ++h) {   // the tile's two page slots
-          const uint32_t sl = 2 * tc.gt + h, slot = sl % nslots;
-          ptx::mbar_wait(bar(empty0, slot), ((sl / nslots) & 1) ^ 1, abort_flag);
-          if (*abort_flag) break;
-          const uint32_t fb = bar(full0, slot);
-          const int pg = 2 * tc.j + h;     // page of the piece in this slot
-          if (tc.j < m.ncache && pg < m.npages) {
-            const int key0 = (tc.ta + pg) * kPage;
-            const int page = __ldg(a.block_table + (size_t)tc.r * a.max_pages + key0 / a.page_size);
+    for (int k = 0; k < kMaxSlots; ++k) last_use[k] = -1;
+    auto bt_chunk = [&](int rr, int base) -> int {
+      const int i = base + lane;
+      return (i < a.max_pages) ? __ldg(a.block_table + (size_t)rr * a.max_pages + i) : -1;
+    };
+    int creq = -1, cbase = 0, cval = -1, nbase = 0, nval = -1;
+    TileCursor tc;
+    tc.init(a);
+    while (__shfl_sync(0xffffffffu, (tc.ok && !*abort_flag) ? 1 : 0, 0)) {
+      const Meta &m = tc.m;
+      bool stop = false;
+      for (int h = 0; h < 2; ++h) {   // the tile's two page slots
+        const uint32_t sl = 2 * tc.gt + h, slot = sl % nslots;
+        if (lane == 0) ptx::mbar_wait(bar(empty0, slot), ((sl / nslots) & 1) ^ 1, abort_flag);
+        stop = __shfl_sync(0xffffffffu, *abort_flag, 0) != 0;
+        if (stop) break;
+        const uint32_t fb = bar(full0, slot);
+        const int pg = 2 * tc.j + h;     // page of the piece in this slot
+        if (tc.j < m.ncache && pg < m.npages) {
+          const int key0 = (tc.ta + pg) * kPage;
+          const int bi = key0 / a.page_size;  // block-table index of the page
+          if (tc.r != creq || bi < cbase || bi >= cbase + 32) {
+            if (tc.r == creq && bi >= nbase && bi < nbase + 32) {
+              cbase = nbase;
+              cval = nval;
+            } else {
+              cbase = bi;
+              cval = bt_chunk(tc.r, cbase);
+            }
+            creq = tc.r;
+            nbase = cbase + 32;
+            nval = bt_chunk(tc.r, nbase);  // the next chunk, ahead of its use
+          }
+          const int page = __shfl_sync(0xffffffffu, cval, bi - cbase);
+          if (lane == 0) {
             int row = oob_row;
             if (page >= 0 && page < a.num_pages) {
               row = ((page * 2 + (is_k ? 0 : 1)) * a.Hkv + tc.g) * a.page_size + key0 % a.page_size;
@@ -412,19 +436,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
             ptx::mbar_arrive_expect_tx(fb, kHalfPageBytes);
             ptx::tma_load_2d_hint(ring(rg0, slot), &tmap_kv, fb, 0, row, stream_policy);
             ptx::tma_load_2d_hint(ring(rg0 + 1, slot), &tmap_kv, fb, 64, row, stream_policy);
-          } else if (tc.j == m.ncache && h == 0) {  // the verify tokens: 16 rows of KV head g
+          }
+        } else if (tc.j == m.ncache && h == 0) {  // the verify tokens: 16 rows of KV head g
+          if (lane == 0) {
             ptx::mbar_arrive_expect_tx(fb, kNewHalfBytes);
             ptx::tma_load_3d(ring(rg0, slot), nmap, fb, 0, tc.g, m.t0);
             ptx::tma_load_3d(ring(rg0 + 1, slot), nmap, fb, 64, tc.g, m.t0);
-          } else {
-            ptx::mbar_arrive(fb);  // empty slot: completes its phase without data
           }
-          last_use[slot] = (int)sl;
+        } else {
+          if (lane == 0) ptx::mbar_arrive(fb);  // empty slot: completes its phase without data
         }
-        tc.advance(a);
+        last_use[slot] = (int)sl;
       }
-      // never leave the CTA with a bulk copy in flight: wait for the latest armed use of every
-      // slot (its phase is the newest one the slot's barrier can complete)
+      if (stop) break;
+      tc.advance(a);
+    }
+    // never leave the CTA with a bulk copy in flight: wait for the latest armed use of every
+    // slot (its phase is the newest one the slot's barrier can complete)
+    if (lane == 0) {
       volatile int no_abort = 0;
       for (int k = 0; k < nslots; ++k)
         if (last_use[k] >= 0)
