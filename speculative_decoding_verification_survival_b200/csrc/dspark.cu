@@ -16,6 +16,7 @@
 #include "calibrate.cuh"
 #include "draft.cuh"
 #include "attn_tc.cuh"
+#include "attn_tk.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -84,6 +85,39 @@ bool encode_new_map(CUtensorMap *map, const void *ptr, int T_cap, int Hkv) {
   cuuint32_t box[3] = {64, 1, (cuuint32_t)tc::kNewRows};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The paged cache as whole-page boxes for the tensor-core kernel: a 4-D view
+// {d 64, row-in-group 8, d-half 2, row group} with strides 256 B, 128 B and 2048 B over the rows
+// of [rows][128] bf16 (rows = pages * 2 * Hkv * page_size, a multiple of 64), 128-byte swizzle,
+// boxes of one page (8 groups): shared memory receives [group][d-half][8 rows][128 B].  Groups
+// past the end read as 0.
+bool encode_kv_page_map(CUtensorMap *map, const void *kv_pages, uint64_t rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {64, 8, 2, rows / 8};
+  cuuint64_t strides[3] = {128 * 2, 64 * 2, 8 * 128 * 2};
+  cuuint32_t box[4] = {64, 8, 2, 8};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(kv_pages), dims,
+             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The verify tokens' own K or V rows [T_cap][Hkv][128] bf16 in the same shared-memory layout: a
+// 4-D view {d 64, token, d-half 2, head} with strides Hkv * 256 B, 128 B and 256 B, 128-byte
+// swizzle, boxes of 8 tokens x both d-halves of one head (one 2048-byte row group); tokens past
+// T_cap read as 0.
+bool encode_new_group_map(CUtensorMap *map, const void *ptr, int T_cap, int Hkv) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {64, (cuuint64_t)T_cap, 2, (cuuint64_t)Hkv};
+  cuuint64_t strides[3] = {(cuuint64_t)Hkv * 128 * 2, 64 * 2, 128 * 2};
+  cuuint32_t box[4] = {64, 8, 2, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides,
              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -218,24 +252,25 @@ int dspark_verify_attn(const void *q, const void *k_new, const void *v_new, cons
   if (dtype == DSPARK_BF16 && D == 128 && page_size % 64 == 0 && kv_rows < (1ull << 31) &&
       K + 1 <= tc::kNewRows && rows_max <= 64) {
     CUtensorMap map, map_kn, map_vn;
-    if (!encode_kv_map(&map, kv_pages, kv_rows) || !encode_new_map(&map_kn, k_new, T_cap, Hkv) ||
-        !encode_new_map(&map_vn, v_new, T_cap, Hkv))
+    if (!encode_kv_page_map(&map, kv_pages, kv_rows) ||
+        !encode_new_group_map(&map_kn, k_new, T_cap, Hkv) ||
+        !encode_new_group_map(&map_vn, v_new, T_cap, Hkv))
       return DSPARK_ECUDA;
-    if (cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tc::kSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(tk::attn_tk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tk::kSmemBytes) != cudaSuccess)
       return DSPARK_ECUDA;
     // programmatic stream serialisation: the kernel's prologue may overlap the previous kernel
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(sms);
-    cfg.blockDim = dim3(tc::kThreads);
-    cfg.dynamicSmemBytes = tc::kSmemBytes;
+    cfg.blockDim = dim3(tk::kThreads);
+    cfg.dynamicSmemBytes = tk::kSmemBytes;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel, map, map_kn, map_vn, a, (int)kv_rows) !=
+    if (cudaLaunchKernelEx(&cfg, tk::attn_tk_kernel, map, map_kn, map_vn, a, (int)kv_rows) !=
         cudaSuccess)
       return DSPARK_ECUDA;
     return launch_status();
