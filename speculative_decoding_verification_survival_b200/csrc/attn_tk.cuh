@@ -18,10 +18,10 @@
 // segment with 33..64 rows is taken in two passes of 32 rows over the same keys (each pass
 // reads its keys again; the schedules of the benchmark workloads give at most 32 rows).
 //
-// Per CTA (384 threads, 12 warps): warps 8 and 11 load K (TMA, one 128-byte-swizzled 4-D box
-// per page, the first and the second page of each tile, a ring of 3 tiles with one barrier
-// each), warp 10 loads V (the same, its own ring), warp 9 issues the MMAs (one thread, polling),
-// warps 0-7 do the softmax and the epilogue: warp w reads the lanes of its
+// Per CTA (384 threads, 12 warps): warp 8 loads K (TMA, one 128-byte-swizzled 4-D box per
+// page, a ring of 3 tiles with one barrier each), warp 10 loads V (the same, its own ring), one
+// thread of warp 9 issues the S^T MMAs and one of warp 11 the P.V MMAs, warps 0-7 do the softmax
+// and the epilogue: warp w reads the lanes of its
 // quadrant q = w % 4 (keys 32q .. 32q + 31 of the tile, and d = 32q .. 32q + 31 of O^T) and the
 // columns of its half hf = w / 4 of the rows, so every thread holds one key's scores for 16
 // rows.  A row's reference maximum comes from the pass's first tile and is raised only when a
@@ -46,7 +46,7 @@ static_assert(kPairsK <= kMaxPairs && kPairsV <= kMaxPairs && 8 * kMaxPairs <= 4
 constexpr int kSoftmaxWarps = 8;
 constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
 constexpr int kWarpK = kSoftmaxWarps, kWarpMma = kSoftmaxWarps + 1, kWarpV = kSoftmaxWarps + 2,
-              kWarpK2 = kSoftmaxWarps + 3;
+              kWarpPV = kSoftmaxWarps + 3;
 constexpr int kThreads = kSoftmaxThreads + 128;
 constexpr int kD = 128;
 constexpr int kNewRows = 16;                         // verify tokens per tile (K + 1 <= 16)
@@ -78,8 +78,8 @@ constexpr int kPS = part_stride(kD);
 // aux region (bytes)
 constexpr uint32_t kBarKFull = 0, kBarSFree = 48, kBarVFull = 64, kBarKEmpty = 128, kBarVEmpty = 192,
                    kBarSFull = 256, kBarPFull = 272, kBarODone = 280, kBarQFull = 288,
-                   kBarQEmpty = 304, kBarOFree = 320, kBarDrain = 328;
-constexpr uint32_t kAuxTmem = 336, kAuxAbort = 340, kAuxLast = 344, kAuxSplit = 352,
+                   kBarQEmpty = 304, kBarOFree = 320, kBarDrain = 328;  // [2]: S^T, P.V issuer
+constexpr uint32_t kAuxTmem = 344, kAuxAbort = 348, kAuxLast = 352, kAuxSplit = 356,
                    kAuxFlags = 384,   // int [2 tile parity][2 halves][4 quadrants]
                    kAuxRmax = 512,    // float [2 tile parity][2 halves][4 quadrants][16 rows]
                    kAuxLsum = 1536;   // float [2 halves][4 quadrants][16 rows]  (to 2048)
@@ -402,6 +402,7 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
     ptx::mbar_init(bar(kBarODone, 0), 1);
     ptx::mbar_init(bar(kBarOFree, 0), kSoftmaxThreads);
     ptx::mbar_init(bar(kBarDrain, 0), 1);
+    ptx::mbar_init(bar(kBarDrain, 1), 1);
     *abort_flag = 0;
     *s_last = 0;
     ptx::fence_mbar_init();
@@ -425,20 +426,15 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
   ptx::grid_dependency_wait();
   ptx::grid_launch_dependents();
 
-  if (warp == kWarpK || warp == kWarpV || warp == kWarpK2) {
+  if (warp == kWarpK || warp == kWarpV) {
     // ------------------------------------------------------------------ TMA producers
-    // A tile (two pages) per ring slot: one barrier per tile, one 4-D box per page.  K, which
-    // the S^T MMAs wait for, comes from two warps (the first and the second page of every tile:
-    // a warp's bulk copies go out one after another), V from one.  The first K warp and the V
-    // warp arm each tile's barrier with the tile's byte count; the second K warp's box completes
-    // its bytes on the same barrier (the transaction count may dip below zero until the arm).
-    // Every producer warp walks the tiles; lane 0 waits on the barriers and issues the copies.
-    // The block-table entries come 32 at a time, lane i holding entry base + i, and the chunk
-    // after the current one is loaded ahead, so a page's lookup is a register shuffle and no
-    // copy waits on a dependent global load.  Tile gt uses tile slot gt mod 3 of its ring.
-    const bool is_k = (warp != kWarpV);
-    const int hsel = (warp == kWarpK) ? 0 : (warp == kWarpK2 ? 1 : -1);  // page(s) this warp loads
-    const bool arms = (hsel != 1);
+    // One warp loads K, another V, a tile (two pages) per ring slot: one barrier and one
+    // transaction count per tile, one 4-D box per page.  The whole warp walks the tiles; lane 0
+    // waits on the barriers and issues the copies.  The block-table entries come 32 at a time,
+    // lane i holding entry base + i, and the chunk after the current one is loaded ahead, so a
+    // page's lookup is a register shuffle and no copy waits on a dependent global load.  Tile gt
+    // uses tile slot gt mod 3 of its ring.
+    const bool is_k = (warp == kWarpK);
     const uint32_t full0 = is_k ? kBarKFull : kBarVFull, empty0 = is_k ? kBarKEmpty : kBarVEmpty;
     const int v = is_k ? 0 : 1;
     const CUtensorMap *nmap = is_k ? &tmap_kn : &tmap_vn;
@@ -488,10 +484,10 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
           pages[h] = (h < npg) ? page_of(tc.p.r, key0[h] / a.page_size) : -1;
         }
         if (lane == 0) {
-          if (arms) ptx::mbar_arrive_expect_tx(fb, (uint32_t)npg * kPageBytes);
+          ptx::mbar_arrive_expect_tx(fb, (uint32_t)npg * kPageBytes);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            if (h < npg && (hsel < 0 || h == hsel)) {
+            if (h < npg) {
               int row = oob_row;
               const int page = pages[h];
               if (page >= 0 && page < a.num_pages) {
@@ -505,7 +501,7 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
           }
         }
       } else {  // the verify tokens: 16 rows of KV head g, two boxes of 8 tokens
-        if (lane == 0 && arms) {
+        if (lane == 0) {
           ptx::mbar_arrive_expect_tx(fb, kNewBytes);
           ptx::tma_load_4d(dst, nmap, fb, 0, m.t0, 0, tc.p.g);
           ptx::tma_load_4d(dst + kGroupBytes, nmap, fb, 0, m.t0 + 8, 0, tc.p.g);
@@ -522,98 +518,90 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
         if (last_use[k] >= 0)
           ptx::mbar_wait(bar(full0, k), ((uint32_t)last_use[k] / npairs) & 1, &no_abort);
     }
-  } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------------ MMA issuer
-    // Two cursors: S^T(js) for the next tile whose K has landed, P.V(jp) for the oldest tile
-    // whose P^T is written.  Whichever is ready is issued (P.V first).  S^T(js) overwrites the
-    // buffer of S^T(js - 2), which the softmax warps release as soon as they have loaded it, so
-    // S^T(j + 2) goes out while the softmax of tile j still runs and, at P^T(j), only P.V(j)
-    // stands between the softmax warps and their next tile.
+  } else if (warp == kWarpMma || warp == kWarpPV) {
+    // ------------------------------------------------------------------ MMA issuers
+    // One thread issues the S^T MMAs (warp 9), another the P.V MMAs (warp 11): each walks the
+    // tiles in order and waits (bounded) on its own barriers, and the two overlap the per-issue
+    // work that surrounds the MMAs.  They touch disjoint tensor memory (S^T buffers, O^T) and
+    // shared memory (K ring and query rows, V ring and P^T); P.V(j) needs P^T(j), which the
+    // softmax warps publish only after loading S^T(j).  S^T(j) overwrites the buffer of
+    // S^T(j - 2), which the softmax warps release as soon as they have loaded it, so S^T(j + 2)
+    // can go out while the softmax of tile j runs.
     if (lane == 0) {
-      TileCursor cs, cp;
-      cs.init(a);
-      cp.init(a);
+      const bool is_s = (warp == kWarpMma);
+      TileCursor c;
+      c.init(a);
       // P^T as B: MN-major with 64-byte swizzle, 8 keys per 512-byte atom
       const uint64_t bd_p = ptx::smem_desc_sw64(pbase, 16, 512);
-      long long idle_since = clock64();
-      while (cp.ok && !*abort_flag) {
-        bool progress = false;
-        if (cp.gt < cs.gt) {
-          const uint32_t pair = cp.gt % kPairsV, ph = (cp.gt / kPairsV) & 1;
-          if ((cp.j > 0 || ptx::mbar_test(bar(kBarOFree, 0), (cp.pq & 1) ^ 1)) &&
-              ptx::mbar_test(bar(kBarPFull, 0), cp.gt & 1) &&
-              ptx::mbar_test(bar(kBarVFull, pair), ph)) {
-            ptx::tc_fence_after();
-            const Meta &m = cp.p.m;
-            const int jj = cp.j;
-            const int ksteps = (jj < m.ncache) ? (min(kTK, m.npages * kPage - jj * kTK) / 16)
-                                               : kNewRows / 16;
-            // V^T as A: MN-major (D on the lanes, d-halves 1024 bytes apart, groups of 8 keys
-            // 2048 apart); fully unrolled k-steps with compile-time descriptor offsets (16 keys:
-            // 4096 bytes of V, 1024 of P^T)
-            const uint64_t ad0 = ptx::smem_desc_sw128(ring(1, pair), 1024, kGroupBytes);
-            const uint32_t acc0 = jj > 0 ? 1u : 0u;
-            if (ksteps == kTK / 16) {
+      uint32_t issued = 0;
+      for (; c.ok; c.advance(a)) {
+        if (is_s) {
+          const uint32_t pair = c.gt % kPairsK, ph = (c.gt / kPairsK) & 1;
+          const int qb = c.pq & 1;
+          if (c.gt >= 2) ptx::mbar_wait(bar(kBarSFree, c.gt & 1), ((c.gt - 2) >> 1) & 1, abort_flag);
+          if (c.j == 0) ptx::mbar_wait(bar(kBarQFull, qb), (c.pq >> 1) & 1, abort_flag);
+          ptx::mbar_wait(bar(kBarKFull, pair), ph, abort_flag);
+          if (*abort_flag) break;
+          ptx::tc_fence_after();
+          const uint32_t d_tmem = tmem + kColS + (c.gt & 1) * kN;
+          // K tile as A (K-major: the keys on the lanes, groups of 8 keys 2048 bytes apart),
+          // the rows as B (K-major); 16 d per k-step: 32 bytes within the 128-byte atom rows,
+          // the d-halves 1024 bytes apart
+          const uint64_t a0 = ptx::smem_desc_sw128(ring(0, pair), 16, kGroupBytes);
+          const uint64_t a1 = ptx::smem_desc_sw128(ring(0, pair) + 1024, 16, kGroupBytes);
+          const uint64_t b0 = ptx::smem_desc_sw128(qbuf(qb, 0), 16, 1024);
+          const uint64_t b1 = ptx::smem_desc_sw128(qbuf(qb, 1), 16, 1024);
 #pragma unroll
-              for (int k = 0; k < kTK / 16; ++k)
-                ptx::mma_bf16_ss(tmem + kColO, ad0 + (uint64_t)(k * 256), bd_p + (uint64_t)(k * 64),
-                                 kIdescPV, k > 0 ? 1u : acc0);
-            } else if (ksteps == kPage / 16) {
-#pragma unroll
-              for (int k = 0; k < kPage / 16; ++k)
-                ptx::mma_bf16_ss(tmem + kColO, ad0 + (uint64_t)(k * 256), bd_p + (uint64_t)(k * 64),
-                                 kIdescPV, k > 0 ? 1u : acc0);
-            } else {
-              ptx::mma_bf16_ss(tmem + kColO, ad0, bd_p, kIdescPV, acc0);
-            }
-            ptx::mma_commit(bar(kBarODone, 0));
-            ptx::mma_commit(bar(kBarVEmpty, pair));
-            cp.advance(a);
-            progress = true;
+          for (int k = 0; k < kD / 16; ++k) {
+            const uint64_t off = (uint64_t)((k & 3) * 2);
+            ptx::mma_bf16_ss(d_tmem, (k < 4 ? a0 : a1) + off, (k < 4 ? b0 : b1) + off, kIdescS,
+                             k > 0 ? 1u : 0u);
           }
-        }
-        if (!progress && cs.ok) {
-          const uint32_t pair = cs.gt % kPairsK, ph = (cs.gt / kPairsK) & 1;
-          const int qb = cs.pq & 1;
-          if ((cs.gt < 2 || ptx::mbar_test(bar(kBarSFree, cs.gt & 1), ((cs.gt - 2) >> 1) & 1)) &&
-              (cs.j > 0 || ptx::mbar_test(bar(kBarQFull, qb), (cs.pq >> 1) & 1)) &&
-              ptx::mbar_test(bar(kBarKFull, pair), ph)) {
-            ptx::tc_fence_after();
-            const uint32_t d_tmem = tmem + kColS + (cs.gt & 1) * kN;
-            // K tile as A (K-major: the keys on the lanes, groups of 8 keys 2048 bytes apart),
-            // the rows as B (K-major); 16 d per k-step: 32 bytes within the 128-byte atom rows,
-            // the d-halves 1024 bytes apart
-            const uint64_t a0 = ptx::smem_desc_sw128(ring(0, pair), 16, kGroupBytes);
-            const uint64_t a1 = ptx::smem_desc_sw128(ring(0, pair) + 1024, 16, kGroupBytes);
-            const uint64_t b0 = ptx::smem_desc_sw128(qbuf(qb, 0), 16, 1024);
-            const uint64_t b1 = ptx::smem_desc_sw128(qbuf(qb, 1), 16, 1024);
+          ptx::mma_commit(bar(kBarSFull, c.gt & 1));
+          ptx::mma_commit(bar(kBarKEmpty, pair));
+          // the pass's last S^T read of its rows: the buffer may be refilled
+          if (c.j == c.p.m.ntiles - 1) ptx::mma_commit(bar(kBarQEmpty, qb));
+        } else {
+          const uint32_t pair = c.gt % kPairsV, ph = (c.gt / kPairsV) & 1;
+          if (c.j == 0) ptx::mbar_wait(bar(kBarOFree, 0), (c.pq & 1) ^ 1, abort_flag);
+          ptx::mbar_wait(bar(kBarPFull, 0), c.gt & 1, abort_flag);
+          ptx::mbar_wait(bar(kBarVFull, pair), ph, abort_flag);
+          if (*abort_flag) break;
+          ptx::tc_fence_after();
+          const Meta &m = c.p.m;
+          const int jj = c.j;
+          const int ksteps = (jj < m.ncache) ? (min(kTK, m.npages * kPage - jj * kTK) / 16)
+                                             : kNewRows / 16;
+          // V^T as A: MN-major (D on the lanes, d-halves 1024 bytes apart, groups of 8 keys
+          // 2048 apart); fully unrolled k-steps with compile-time descriptor offsets (16 keys:
+          // 4096 bytes of V, 1024 of P^T)
+          const uint64_t ad0 = ptx::smem_desc_sw128(ring(1, pair), 1024, kGroupBytes);
+          const uint32_t acc0 = jj > 0 ? 1u : 0u;
+          if (ksteps == kTK / 16) {
 #pragma unroll
-            for (int k = 0; k < kD / 16; ++k) {
-              const uint64_t off = (uint64_t)((k & 3) * 2);
-              ptx::mma_bf16_ss(d_tmem, (k < 4 ? a0 : a1) + off, (k < 4 ? b0 : b1) + off, kIdescS,
-                               k > 0 ? 1u : 0u);
-            }
-            ptx::mma_commit(bar(kBarSFull, cs.gt & 1));
-            ptx::mma_commit(bar(kBarKEmpty, pair));
-            // the pass's last S^T read of its rows: the buffer may be refilled
-            if (cs.j == cs.p.m.ntiles - 1) ptx::mma_commit(bar(kBarQEmpty, qb));
-            cs.advance(a);
-            progress = true;
+            for (int k = 0; k < kTK / 16; ++k)
+              ptx::mma_bf16_ss(tmem + kColO, ad0 + (uint64_t)(k * 256), bd_p + (uint64_t)(k * 64),
+                               kIdescPV, k > 0 ? 1u : acc0);
+          } else if (ksteps == kPage / 16) {
+#pragma unroll
+            for (int k = 0; k < kPage / 16; ++k)
+              ptx::mma_bf16_ss(tmem + kColO, ad0 + (uint64_t)(k * 256), bd_p + (uint64_t)(k * 64),
+                               kIdescPV, k > 0 ? 1u : acc0);
+          } else {
+            ptx::mma_bf16_ss(tmem + kColO, ad0, bd_p, kIdescPV, acc0);
           }
+          ptx::mma_commit(bar(kBarODone, 0));
+          ptx::mma_commit(bar(kBarVEmpty, pair));
         }
-        if (progress) {
-          idle_since = clock64();
-        } else if (clock64() - idle_since > ptx::kWaitLimitCycles) {
-          *abort_flag = 1;
-          raise_error(DSPARK_DERR_TIMEOUT);
-        }
+        ++issued;
       }
       // every MMA this thread issued has completed before the CTA releases shared memory and
-      // TMEM, also after an abort
-      if (cs.gt > 0 || cp.gt > 0) {
-        ptx::mma_commit(bar(kBarDrain, 0));
+      // TMEM, also after an abort (each issuer drains through its own barrier)
+      if (issued > 0) {
+        const uint32_t drain = bar(kBarDrain, is_s ? 0 : 1);
+        ptx::mma_commit(drain);
         volatile int no_abort = 0;
-        ptx::mbar_wait(bar(kBarDrain, 0), 0, &no_abort);
+        ptx::mbar_wait(drain, 0, &no_abort);
       }
     }
   } else {
