@@ -15,7 +15,6 @@
 #include "kv_commit.cuh"
 #include "calibrate.cuh"
 #include "draft.cuh"
-#include "attn_tc.cuh"
 #include "attn_tk.cuh"
 
 #include <cudaTypedefs.h>
@@ -59,34 +58,6 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   }
   return fn;
-}
-
-// The paged cache viewed as a 2-D bf16 tensor [rows][128], rows = pages * 2 * Hkv * page_size;
-// boxes of 64 rows x 64 elements (128 B) with 128-byte swizzle, out-of-range rows read as 0.
-bool encode_kv_map(CUtensorMap *map, const void *kv_pages, uint64_t rows) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {128, rows};
-  cuuint64_t strides[1] = {128 * 2};
-  cuuint32_t box[2] = {64, 64};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(kv_pages), dims,
-             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// The verify tokens' own K or V rows [T_cap][Hkv][128] bf16 as a 3-D tensor; boxes of
-// 16 tokens x 1 head x 64 elements (128 B) with 128-byte swizzle, tokens past T_cap read as 0.
-bool encode_new_map(CUtensorMap *map, const void *ptr, int T_cap, int Hkv) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {128, (cuuint64_t)Hkv, (cuuint64_t)T_cap};
-  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)Hkv * 128 * 2};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)tc::kNewRows};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
-             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // The paged cache as whole-page boxes for the tensor-core kernel: a 4-D view
@@ -250,7 +221,7 @@ int dspark_verify_attn(const void *q, const void *k_new, const void *v_new, cons
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const uint64_t kv_rows = (uint64_t)num_pages * 2 * Hkv * page_size;
   if (dtype == DSPARK_BF16 && D == 128 && page_size % 64 == 0 && kv_rows < (1ull << 31) &&
-      K + 1 <= tc::kNewRows && rows_max <= 64) {
+      K + 1 <= tk::kNewRows && rows_max <= 64) {
     CUtensorMap map, map_kn, map_vn;
     if (!encode_kv_page_map(&map, kv_pages, kv_rows) ||
         !encode_new_group_map(&map_kn, k_new, T_cap, Hkv) ||
