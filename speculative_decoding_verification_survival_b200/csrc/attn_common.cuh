@@ -31,14 +31,16 @@ struct AttnPlanHeader {
   float tc_bound;        // the largest modelled CTA cost of those ranges
 };
 
-// Cost model of the tensor-core kernel's work, in units of one 64-key cache page (fitted to a
-// per-CTA trace: 1.37 us per 128-key tile, 2.4 us per piece, 3.6 us per merge of split
-// partials).  A segment's verify tokens are one tile, its epilogue and the pipeline refill of
-// the next piece a piece cost; the head piece of a split segment usually merges, as the next
-// CTA finishes the segment's rest first.
-constexpr float kCostNewTile = 2.0f;
-constexpr float kCostPiece = 3.5f;
-constexpr float kCostMerge = 5.25f;
+// Cost model of the tensor-core kernel's work, in units of one 64-key cache page (about 0.75 us
+// of a CTA's time at full clock).  A segment's verify tokens and its query rows cost 5, a piece
+// (its epilogue, about 4 us, and the refill of the pipeline for the next piece) 10, merging the
+// partials of a split segment 8: the middle of the plateau of a sweep of the three constants,
+// timed on workloads of 64 to 1024 requests (the per-CTA finish times of one call put a piece
+// near 9 pages).  The head piece of a split segment usually merges, as the next CTA finishes the
+// segment's rest first.
+constexpr float kCostNewTile = 5.0f;
+constexpr float kCostPiece = 10.0f;
+constexpr float kCostMerge = 8.0f;
 // Candidate cost bounds the plan tests at once (one per thread of its single CTA).
 constexpr int kPlanThreads = 1024;
 
@@ -106,7 +108,7 @@ __device__ __forceinline__ void find_segment(const int *__restrict__ tile_prefix
 // Greedy fill of CTAs in unit order under a cost bound: a segment goes whole into the current
 // CTA if it fits; otherwise the CTA takes a head piece of an even number of cache pages (at
 // least 2, with the piece and merge costs) and the rest continues in the next CTAs (which may
-// cut it again).  A range boundary never falls inside a segment's verify-token units.  Returns
+// cut it again); a bound under which not even a two-page piece fits counts as infeasible.  A range boundary never falls inside a segment's verify-token units.  Returns
 // the number of CTAs used (stops counting past `cap`); when `begin` is given, records the first
 // unit of every CTA used (begin[0] = 0).
 __device__ int plan_fill(const int *__restrict__ tile_prefix, int R, int Hkv, float bound,
@@ -132,8 +134,8 @@ __device__ int plan_fill(const int *__restrict__ tile_prefix, int R, int Hkv, fl
         const float rest = (float)(u - done) + kCostNewTile + kCostPiece;
         if (rest <= bound || used > cap) { cur = rest; break; }
         // a segment cut from its start here (no head piece placed above) has its head now
-        int mid = (int)floorf(bound - kCostPiece - (done == 0 ? kCostMerge : 0.f)) & ~1;
-        mid = max(mid, 2);
+        const int mid = (int)floorf(bound - kCostPiece - (done == 0 ? kCostMerge : 0.f)) & ~1;
+        if (mid < 2) return cap + 1;  // not even a two-page piece fits: the bound is infeasible
         done = min(u, done + mid);
       }
     }
