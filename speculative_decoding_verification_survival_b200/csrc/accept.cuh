@@ -73,7 +73,7 @@ __device__ __forceinline__ float exp2_sfu(float x) {
 // The scale c = log2(e) / tau as an unevaluated float sum hi + lo (lo = c - hi rounded), and in
 // float64 for the few per-request evaluations done at that precision.
 struct ExpScale {
-  float hi, lo;
+  float hi, lo;  // hi = c rounded toward zero, lo = c - hi rounded (> 0 for sampled rows)
   double d;
   // d * c in float32 without the systematic error of a rounded c.  d = -inf (a masked logit,
   // or padding) is first clamped to a large finite negative number, whose 2^x is still 0:
@@ -108,6 +108,80 @@ __device__ __forceinline__ void cvt8(const Raw8<__nv_bfloat16> &r, float (&v)[8]
 __device__ __forceinline__ void cvt8(const Raw8<float> &r, float (&v)[8]) {
   v[0] = r.a.x; v[1] = r.a.y; v[2] = r.a.z; v[3] = r.a.w;
   v[4] = r.b.x; v[5] = r.b.y; v[6] = r.b.z; v[7] = r.b.w;
+}
+
+// bf16 logits, sampled verification: this thread's share of one row (16-byte groups g = tid,
+// tid + 256, ...) as a running maximum m and Z = sum 2^((z - m) c), with as few instructions per
+// element as the arithmetic allows (the pass is issue-bound before it is memory-bound on this
+// part).  A pair of groups' maximum comes from packed bf16 pairs and Z is rescaled only when it
+// rises; per pair of elements the bf16 -> float conversion is a shift and a mask, then
+// d = z - m (exact), d hi + d lo and the running sums run as packed float pairs, and ex2 per
+// element: the even and the odd elements of a pair of groups each go to one float partial (8
+// terms each), the partials summed in float64.  Loads run one step of two groups ahead, in two
+// register sets used in turn.
+using ptx::f2_add;
+using ptx::f2_fma;
+using ptx::f2_mul;
+using ptx::f2_pack;
+using ptx::f2_unpack;
+__device__ __forceinline__ uint64_t f2_pack_dup(float x) { return ptx::f2_pack(x, x); }
+__device__ __forceinline__ float bf16_lo_f(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi_f(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+  const __nv_bfloat162 r = __hmax2(*reinterpret_cast<const __nv_bfloat162 *>(&a),
+                                   *reinterpret_cast<const __nv_bfloat162 *>(&b));
+  return *reinterpret_cast<const uint32_t *>(&r);
+}
+__device__ __forceinline__ void stats_bf16_sampled(const uint4 *__restrict__ rowv, int nv,
+                                                   const ExpScale &c, float &m, double &Z) {
+  const int tid = threadIdx.x;
+  const uint64_t hi2 = f2_pack_dup(c.hi), lo2 = f2_pack_dup(c.lo);
+  // a pair of groups: its maximum, the rescale if it rises, its 16 terms
+  auto step = [&](const uint4 &a, const uint4 &b) {
+    const uint32_t p = bmax2(bmax2(bmax2(a.x, a.y), bmax2(a.z, a.w)),
+                             bmax2(bmax2(b.x, b.y), bmax2(b.z, b.w)));
+    const float gm = fmaxf(bf16_lo_f(p), bf16_hi_f(p));
+    if (gm > m) {
+      if (m != -INFINITY) Z *= exp2(((double)m - (double)gm) * c.d);
+      m = gm;
+    }
+    if (m == -INFINITY) return;  // every value so far is -inf
+    const uint64_t nm2 = f2_pack_dup(-m);
+    uint64_t s2 = 0;  // (even, odd) partial sums: two float zeros
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint64_t d2 = f2_add(f2_pack(bf16_lo_f(w[i]), bf16_hi_f(w[i])), nm2);
+      const uint64_t e2 = f2_fma(d2, lo2, f2_mul(d2, hi2));
+      float e0, e1;
+      f2_unpack(e2, e0, e1);
+      s2 = f2_add(s2, f2_pack(exp2_sfu(e0), exp2_sfu(e1)));
+    }
+    float s0, s1;
+    f2_unpack(s2, s0, s1);
+    Z += (double)(s0 + s1);
+  };
+  constexpr int kPair = 2 * kAccThreads;  // groups per step of the whole CTA
+  const int steps = nv / kPair;           // steps in which every thread has both groups
+  uint4 a0, b0, a1, b1;
+  if (steps > 0) { a0 = __ldg(rowv + tid); b0 = __ldg(rowv + tid + kAccThreads); }
+  int s = 0;
+  for (; s + 1 < steps; s += 2) {
+    const int g1 = (s + 1) * kPair + tid;
+    a1 = __ldg(rowv + g1);
+    b1 = __ldg(rowv + g1 + kAccThreads);
+    step(a0, b0);
+    if (s + 2 < steps) {
+      const int g2 = (s + 2) * kPair + tid;
+      a0 = __ldg(rowv + g2);
+      b0 = __ldg(rowv + g2 + kAccThreads);
+    }
+    step(a1, b1);
+  }
+  if (s < steps) step(a0, b0);
+  // the rest: single groups (the other of a pair is all -inf)
+  const uint4 ninf = make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+  for (int g = steps * kPair + tid; g < nv; g += kAccThreads) step(__ldg(rowv + g), ninf);
 }
 
 // One CTA per scheduled logit row: one streaming pass with 16-byte loads, 32 elements per thread
@@ -171,7 +245,15 @@ accept_stats_kernel(const T *__restrict__ target, const T *__restrict__ draft, i
   };
   const bool vec = ((reinterpret_cast<uintptr_t>(row) & 15) == 0) && (V % 8 == 0) &&
                    (sizeof(T) == 2 || (reinterpret_cast<uintptr_t>(row) & 31) == 0);
-  if (vec) {
+  bool done = false;
+  if constexpr (sizeof(T) == 2 && !GREEDY) {
+    if (vec) {
+      stats_bf16_sampled(reinterpret_cast<const uint4 *>(row), V / 8, c, m, Z);
+      done = true;
+    }
+  }
+  if (done) {
+  } else if (vec) {
     // the next step's loads are issued before this step's values are used, so every thread
     // keeps loads in flight while it computes
     constexpr int kU = 2;

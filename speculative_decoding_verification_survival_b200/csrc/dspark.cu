@@ -285,8 +285,12 @@ int dspark_accept(const void *target_logits, const void *draft_logits, int dtype
   if (!ws || ws_bytes < accept_ws_bytes(R, K, T_cap) || !aligned16(ws)) return DSPARK_EWORKSPACE;
   ExpScale c;
   c.d = greedy ? 0.0 : 1.4426950408889634 / (double)temperature;
+  // hi rounded toward zero, so lo >= 0 (and > 0: a zero lo is replaced by the least normal
+  // float), which lets d * hi + d * lo stay -inf for a -inf logit without a clamp
   c.hi = (float)c.d;
-  c.lo = (float)(c.d - (double)c.hi);
+  if ((double)c.hi > c.d) c.hi = std::nextafter(c.hi, 0.f);  // c > 0: toward zero
+  if (greedy) c.hi = 0.f;
+  c.lo = greedy ? 0.f : fmaxf((float)(c.d - (double)c.hi), 1.17549435e-38f);
   RowStats *st = static_cast<RowStats *>(ws);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int nrows = T_cap + R * K;
