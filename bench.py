@@ -125,23 +125,21 @@ class ClockSampler:
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch, from an ncu
-# capture, keyed by the SHA-1 of the kernel sources the capture ran; any change to those
-# sources voids the figure.  A workload too large to capture is captured on a smaller case of
-# the same kernel and scaled by algorithmic bytes: (sha, bytes, algorithmic bytes of the capture)
-NCU_TRAFFIC = {
-    # 626.618624 MB read + 4.616192 MB written, 621 088 768 algorithmic bytes
-    "qwen3-4b-64req": ("b7667a45921c3d9cfd3c89a9121bfc2c701ef656", 631234816, 621088768),
-}
+# capture, keyed by the SHA-1 of the sources the attention kernel is built from (ATTN_SOURCES);
+# any change to those voids the figure.  Entries: (sha, bytes, algorithmic bytes of the capture);
+# a capture of another size of the same workload is scaled by algorithmic bytes.
+NCU_TRAFFIC = {}
+
+ATTN_SOURCES = ("attn_tk.cuh", "attn_common.cuh", "ptx_sm100.cuh", "common.cuh", "dspark.cu")
 
 
 def kernel_source_hash():
     import hashlib
     d = os.path.join(ROOT, "speculative_decoding_verification_survival_b200", "csrc")
     h = hashlib.sha1()
-    for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(d, name), "rb") as fh:
-                h.update(name.encode() + b"\0" + fh.read())
+    for name in ATTN_SOURCES:
+        with open(os.path.join(d, name), "rb") as fh:
+            h.update(name.encode() + b"\0" + fh.read())
     return h.hexdigest()
 
 

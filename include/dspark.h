@@ -165,7 +165,7 @@ size_t dspark_verify_attn_workspace_bytes(int R, int Hq, int Hkv, int D, int K);
  * the largest modelled cost of a range: one per 64-key page, five for a segment's verify
  * tokens and query rows, ten per piece (a segment cut by range boundaries is computed in pieces)
  * and eight for merging a cut segment's partials; boundaries fall on even page counts and never inside a
- * segment's verify-token units.  It runs a greedy fill for 1024 candidate bounds at once.
+ * segment's verify-token units.  It runs the greedy fill for 1024 candidate bounds at once.
  * It also records, per request, the flattened offset, the token count and whether the
  * flattening is well formed (1 <= Q_r <= K + 1 tokens inside [0, T_cap), token j carrying the
  * marker (r, kv_len[r] + j)); a malformed request sets DSPARK_DERR_OFFSETS / _MARKER here and

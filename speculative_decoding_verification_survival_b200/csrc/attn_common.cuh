@@ -42,7 +42,9 @@ constexpr float kCostNewTile = 5.0f;
 constexpr float kCostPiece = 10.0f;
 constexpr float kCostMerge = 8.0f;
 // Candidate cost bounds the plan tests at once (one per thread of its single CTA).
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanCandidates = 1024;
+// Requests whose segment costs the plan keeps in shared memory (more go to the workspace).
+constexpr int kPlanSmemRequests = 8192;
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -57,6 +59,7 @@ struct AttnWs {
   int4 *cta_start;   // [max_ctas]: first segment of tensor-core CTA c {r, g, s0, units}, r < 0: none
   int *cta_begin;    // [max_ctas + 1]: first unit of tensor-core CTA c; [tc_ctas] = total
   float *partials;   // [2 * max_ctas][rows_max][part_stride(D)]: acc[D], m, l per row
+  float *seg_cost;   // [R]: modelled cost of a whole segment of request r (plan scratch)
 };
 
 __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, int D,
@@ -70,6 +73,7 @@ __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, i
   const size_t o_beg = off;                off += align256((size_t)(max_ctas + 1) * sizeof(int));
   const size_t o_par = off;
   off += align256((size_t)2 * max_ctas * rows_max * part_stride(D) * sizeof(float));
+  const size_t o_sc = off;                 off += align256((size_t)R * sizeof(float));
   if (ws) {
     char *b = static_cast<char *>(base);
     ws->hdr = reinterpret_cast<AttnPlanHeader *>(b + o_hdr);
@@ -79,6 +83,7 @@ __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, i
     ws->cta_start = reinterpret_cast<int4 *>(b + o_cst);
     ws->cta_begin = reinterpret_cast<int *>(b + o_beg);
     ws->partials = reinterpret_cast<float *>(b + o_par);
+    ws->seg_cost = reinterpret_cast<float *>(b + o_sc);
   }
   return off;
 }
@@ -111,18 +116,24 @@ __device__ __forceinline__ void find_segment(const int *__restrict__ tile_prefix
 // cut it again); a bound under which not even a two-page piece fits counts as infeasible.  A range boundary never falls inside a segment's verify-token units.  Returns
 // the number of CTAs used (stops counting past `cap`); when `begin` is given, records the first
 // unit of every CTA used (begin[0] = 0).
-__device__ int plan_fill(const int *__restrict__ tile_prefix, int R, int Hkv, float bound,
-                         int cap, int *begin) {
+__device__ int plan_fill(const int *__restrict__ tile_prefix, const float *seg_cost, int R, int Hkv,
+                         float bound, int cap, int *begin) {
   int used = 1;
   float cur = 0.f;
   if (begin) begin[0] = 0;
   for (int r = 0; r < R && used <= cap; ++r) {
-    const int seg_units = (tile_prefix[r + 1] - tile_prefix[r]) / Hkv;
-    const int u = seg_units - kSegTail;
+    // a segment's cost when whole: its cache pages, its verify tokens and one piece
+    const float full = seg_cost[r];
+    const float all = (float)Hkv * full;
+    if (cur + all <= bound) {  // the request's Hkv segments all fit: the usual case
+      cur += all;
+      continue;
+    }
+    const int u = (int)(full - kCostNewTile - kCostPiece);  // cache pages of a segment
+    const int seg_units = u + kSegTail;
     for (int g = 0; g < Hkv && used <= cap; ++g) {
-      const int s0 = tile_prefix[r] + g * seg_units;
-      const float full = (float)u + kCostNewTile + kCostPiece;
       if (cur + full <= bound) { cur += full; continue; }
+      const int s0 = tile_prefix[r] + g * seg_units;
       int done = 0;  // cache pages of this segment placed in earlier CTAs
       int head = (int)floorf(bound - cur - kCostPiece - kCostMerge);
       head &= ~1;
@@ -221,7 +232,7 @@ attn_plan_kernel(const int32_t *__restrict__ kv_len, const int32_t *__restrict__
   seg_max = warp_max(seg_max);
   __shared__ float s_part[32], s_pmax[32];
   if (lane == 0) { s_part[warp] = mine; s_pmax[warp] = seg_max; }
-  if (tid == 0) s_best = kPlanThreads;
+  if (tid == 0) s_best = kPlanCandidates;
   __syncthreads();
   if (tid == 0) {
     float t = 0.f, mx = 0.f;
@@ -230,14 +241,29 @@ attn_plan_kernel(const int32_t *__restrict__ kv_len, const int32_t *__restrict__
     s_pmax[0] = mx;
   }
   __syncthreads();
+  // Each of the first kPlanCandidates threads runs the greedy fill for one candidate bound in
+  // (lo, hi] (hi always fits), reading the segment costs from shared memory; the smallest that
+  // needs at most tc_ctas CTAs wins and its fill is run once more to record where each CTA
+  // starts.
   const float lo = s_tot / (float)tc_ctas;
   const float hi = lo + s_pmax[0] + kCostMerge + kCostPiece;
-  const float bound = lo + (hi - lo) * (float)(tid + 1) / (float)blockDim.x;
-  if (plan_fill(ws.tile_prefix, R, Hkv, bound, tc_ctas, nullptr) <= tc_ctas) atomicMin(&s_best, tid);
+  __shared__ float s_cost[kPlanSmemRequests];
+  const bool staged = R <= kPlanSmemRequests;
+  float *cost = staged ? s_cost : ws.seg_cost;
+  for (int r = tid; r < R; r += blockDim.x)
+    cost[r] = (float)((ws.tile_prefix[r + 1] - ws.tile_prefix[r]) / Hkv - kSegTail) +
+              kCostNewTile + kCostPiece;
   __syncthreads();
-  const int best = min(s_best, (int)blockDim.x - 1);
-  if (tid == best) {
-    const int used = plan_fill(ws.tile_prefix, R, Hkv, bound, tc_ctas, ws.cta_begin);
+  if (tid < kPlanCandidates) {
+    const float cand = lo + (hi - lo) * (float)(tid + 1) / (float)kPlanCandidates;
+    if (plan_fill(ws.tile_prefix, cost, R, Hkv, cand, tc_ctas, nullptr) <= tc_ctas)
+      atomicMin(&s_best, tid);
+  }
+  __syncthreads();
+  const float bound = lo + (hi - lo) * (float)(min(s_best, kPlanCandidates - 1) + 1) /
+                               (float)kPlanCandidates;
+  if (tid == 0) {
+    const int used = plan_fill(ws.tile_prefix, cost, R, Hkv, bound, tc_ctas, ws.cta_begin);
     // trailing CTAs get empty ranges; had no bound fitted, the last CTA would take the rest
     for (int c = min(used, tc_ctas); c <= tc_ctas; ++c) ws.cta_begin[c] = total;
     ws.hdr->tc_bound = bound;
