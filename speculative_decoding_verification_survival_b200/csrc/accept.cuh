@@ -117,8 +117,9 @@ __device__ __forceinline__ void cvt8(const Raw8<float> &r, float (&v)[8]) {
 // rises; per pair of elements the bf16 -> float conversion is a shift and a mask, then
 // d = z - m (exact), d hi + d lo and the running sums run as packed float pairs, and ex2 per
 // element: the even and the odd elements of a pair of groups each go to one float partial (8
-// terms each), the partials summed in float64.  Loads run one step of two groups ahead, in two
-// register sets used in turn.
+// terms each), the partials summed in float64.  Loads run one step of four groups ahead (64
+// bytes per thread in flight; four CTAs per SM, so 64 KB per SM), in two register sets used in
+// turn.
 using ptx::f2_add;
 using ptx::f2_fma;
 using ptx::f2_mul;
@@ -161,27 +162,33 @@ __device__ __forceinline__ void stats_bf16_sampled(const uint4 *__restrict__ row
     f2_unpack(s2, s0, s1);
     Z += (double)(s0 + s1);
   };
-  constexpr int kPair = 2 * kAccThreads;  // groups per step of the whole CTA
-  const int steps = nv / kPair;           // steps in which every thread has both groups
-  uint4 a0, b0, a1, b1;
-  if (steps > 0) { a0 = __ldg(rowv + tid); b0 = __ldg(rowv + tid + kAccThreads); }
+  // a step is two pairs of groups per thread (four 16-byte loads); the next step's loads are
+  // issued before this step's values are used, in two register sets used in turn
+  constexpr int kStep = 4 * kAccThreads;  // groups per step of the whole CTA
+  const int steps = nv / kStep;           // steps in which every thread has all four groups
+  uint4 x0[4], x1[4];
+  auto load = [&](uint4 (&x)[4], int st) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] = __ldg(rowv + st * kStep + u * kAccThreads + tid);
+  };
+  if (steps > 0) load(x0, 0);
   int s = 0;
   for (; s + 1 < steps; s += 2) {
-    const int g1 = (s + 1) * kPair + tid;
-    a1 = __ldg(rowv + g1);
-    b1 = __ldg(rowv + g1 + kAccThreads);
-    step(a0, b0);
-    if (s + 2 < steps) {
-      const int g2 = (s + 2) * kPair + tid;
-      a0 = __ldg(rowv + g2);
-      b0 = __ldg(rowv + g2 + kAccThreads);
-    }
-    step(a1, b1);
+    load(x1, s + 1);
+    step(x0[0], x0[1]);
+    step(x0[2], x0[3]);
+    if (s + 2 < steps) load(x0, s + 2);
+    step(x1[0], x1[1]);
+    step(x1[2], x1[3]);
   }
-  if (s < steps) step(a0, b0);
+  if (s < steps) {
+    step(x0[0], x0[1]);
+    step(x0[2], x0[3]);
+  }
+  const int done_groups = steps * kStep;
   // the rest: single groups (the other of a pair is all -inf)
   const uint4 ninf = make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
-  for (int g = steps * kPair + tid; g < nv; g += kAccThreads) step(__ldg(rowv + g), ninf);
+  for (int g = done_groups + tid; g < nv; g += kAccThreads) step(__ldg(rowv + g), ninf);
 }
 
 // One CTA per scheduled logit row: one streaming pass with 16-byte loads, 32 elements per thread
@@ -189,7 +196,7 @@ __device__ __forceinline__ void stats_bf16_sampled(const uint4 *__restrict__ row
 // need the maximum and its lowest index.  Five CTAs per SM (registers capped to fit), so that a
 // 64-request step's 704 rows run as one wave of 740 rather than 1.2 waves of 592.
 template <typename T, bool GREEDY>
-__global__ void __launch_bounds__(kAccThreads, 5)
+__global__ void __launch_bounds__(kAccThreads, (sizeof(T) == 2 && !GREEDY) ? 4 : 5)
 accept_stats_kernel(const T *__restrict__ target, const T *__restrict__ draft, int V, int R, int K,
                     int T_cap, const int32_t *__restrict__ verify_len,
                     const int32_t *__restrict__ q_offsets, ExpScale c,
