@@ -723,11 +723,21 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
       // through shared memory.  O^T: this thread's lane is d = kk, its columns its rows.
       float *ls = lsum_buf + hf * 4 * kRH;
       if (m.ntiles > 0) {
+        // the 16 sums over the warp's lanes by halving exchanges (16 shuffles, not 80): at each
+        // level a lane keeps one half of its values and adds the partner's copy of that half;
+        // every sum takes the same pairs as a butterfly warp sum.  Row i ends in lanes 2i, 2i + 1.
 #pragma unroll
-        for (int i = 0; i < kRH; ++i) {
-          const float v = warp_sum(lpart[i]);
-          if (lane == i) ls[q * kRH + i] = v;
+        for (int w = kRH / 2, bit = 16; w >= 1; w >>= 1, bit >>= 1) {
+          const bool up = (lane & bit) != 0;
+#pragma unroll
+          for (int k = 0; k < w; ++k) {
+            const float send = up ? lpart[k] : lpart[k + w];
+            const float keep = up ? lpart[k + w] : lpart[k];
+            lpart[k] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+          }
         }
+        lpart[0] += __shfl_xor_sync(0xffffffffu, lpart[0], 1);
+        if ((lane & 1) == 0) ls[q * kRH + (lane >> 1)] = lpart[0];
         ptx::mbar_wait(bar(kBarODone, 0), (gt + m.ntiles - 1) & 1, abort_flag);
         ptx::tc_fence_after();
       }
@@ -749,14 +759,18 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
         ptx::tmem_wait_ld();
         ptx::tc_fence_before();
         ptx::mbar_arrive(bar(kBarOFree, 0));  // O^T read: the next pass's P.V may overwrite it
+        // rows r0 + 16 hf + i: token jt, head ih of the group, stepped without dividing
+        int jt = (r0 + hf * kRH) / G, ih = (r0 + hf * kRH) % G;
 #pragma unroll
         for (int i = 0; i < kRH; ++i) {
           const int rl = hf * kRH + i;
           if (rl < nr) {
             const float l = ls[i] + ls[kRH + i] + ls[2 * kRH + i] + ls[3 * kRH + i];
-            const int rr = r0 + rl, jt = rr / G, ih = rr % G;
+            const int rr = r0 + rl;
             if (whole) {
-              og[((size_t)(m.t0 + jt) * a.Hq + g * G + ih) * kD + kk] = __float2bfloat16_rn(o[i] / l);
+              og[((size_t)(m.t0 + jt) * a.Hq + g * G + ih) * kD + kk] =
+                  // l >= 1: the row's reference maximum is one of its own scores
+                  __float2bfloat16_rn(__fdividef(o[i], l));
             } else {
               part[(size_t)rr * kPS + kk] = o[i];
               if (kk == 0) {
@@ -764,6 +778,10 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
                 part[(size_t)rr * kPS + kD + 1] = l;
               }
             }
+          }
+          if (++ih == G) {
+            ih = 0;
+            ++jt;
           }
         }
         gt += m.ntiles;
