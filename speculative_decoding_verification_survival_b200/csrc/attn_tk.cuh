@@ -759,29 +759,45 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
         ptx::tmem_wait_ld();
         ptx::tc_fence_before();
         ptx::mbar_arrive(bar(kBarOFree, 0));  // O^T read: the next pass's P.V may overwrite it
-        // rows r0 + 16 hf + i: token jt, head ih of the group, stepped without dividing
-        int jt = (r0 + hf * kRH) / G, ih = (r0 + hf * kRH) % G;
+        if (whole) {
+          // the pass's output rows as bf16 [32 rows][128 d] in the P^T buffer (free: the last
+          // P.V has completed, the next pass's first P^T comes after two barriers), then 16-byte
+          // stores of whole rows: row rl is token (r0 + rl) / G, head (r0 + rl) % G of the group
 #pragma unroll
-        for (int i = 0; i < kRH; ++i) {
-          const int rl = hf * kRH + i;
-          if (rl < nr) {
+          for (int i = 0; i < kRH; ++i) {
+            const int rl = hf * kRH + i;
             const float l = ls[i] + ls[kRH + i] + ls[2 * kRH + i] + ls[3 * kRH + i];
-            const int rr = r0 + rl;
-            if (whole) {
-              og[((size_t)(m.t0 + jt) * a.Hq + g * G + ih) * kD + kk] =
-                  // l >= 1: the row's reference maximum is one of its own scores
-                  __float2bfloat16_rn(__fdividef(o[i], l));
-            } else {
+            // l >= 1 (a visible row): its reference maximum is one of its own scores
+            const __nv_bfloat16 v = __float2bfloat16_rn(rl < nr ? __fdividef(o[i], l) : 0.f);
+            asm volatile("st.shared.b16 [%0], %1;" ::"r"(pbase + (uint32_t)(rl * kD + kk) * 2u),
+                         "h"(*reinterpret_cast<const unsigned short *>(&v))
+                         : "memory");
+          }
+          ptx::named_bar_sync(kBarAllSoftmax, kSoftmaxThreads);
+#pragma unroll
+          for (int c = tid; c < kN * (kD / 8); c += kSoftmaxThreads) {
+            const int rl = c / (kD / 8), ch = c % (kD / 8);
+            if (rl < nr) {
+              const uint4 w = ptx::ld_shared_v4(pbase + (uint32_t)(rl * kD + ch * 8) * 2u);
+              const int rr = r0 + rl, jt = rr / G, ih = rr % G;
+              *reinterpret_cast<uint4 *>(og + ((size_t)(m.t0 + jt) * a.Hq + g * G + ih) * kD +
+                                         ch * 8) = w;
+            }
+          }
+          ptx::named_bar_sync(kBarAllSoftmax, kSoftmaxThreads);
+        } else {
+#pragma unroll
+          for (int i = 0; i < kRH; ++i) {
+            const int rl = hf * kRH + i;
+            if (rl < nr) {
+              const float l = ls[i] + ls[kRH + i] + ls[2 * kRH + i] + ls[3 * kRH + i];
+              const int rr = r0 + rl;
               part[(size_t)rr * kPS + kk] = o[i];
               if (kk == 0) {
                 part[(size_t)rr * kPS + kD] = mref[i];
                 part[(size_t)rr * kPS + kD + 1] = l;
               }
             }
-          }
-          if (++ih == G) {
-            ih = 0;
-            ++jt;
           }
         }
         gt += m.ntiles;
