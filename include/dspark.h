@@ -162,9 +162,9 @@ size_t dspark_verify_attn_workspace_bytes(int R, int Hq, int Hkv, int D, int K);
  * contributing Hkv * (ceil(kv_len[r] / 64) + 8) units (its 64-key cache tiles, then eight
  * units standing for its own verify tokens and the segment's epilogue).  The plan splits it
  * into contiguous ranges, one per persistent CTA of the tensor-core kernel, chosen to minimise
- * the largest modelled cost of a range: one per 64-key page, five for a segment's verify
- * tokens and query rows, ten per piece (a segment cut by range boundaries is computed in pieces)
- * and eight for merging a cut segment's partials; boundaries fall on even page counts and never inside a
+ * the largest modelled cost of a range: one per 64-key page, four for a segment's verify
+ * tokens and query rows, seven per piece (a segment cut by range boundaries is computed in
+ * pieces) and six for merging a cut segment's partials; boundaries fall on even page counts and never inside a
  * segment's verify-token units.  It runs the greedy fill for 1024 candidate bounds at once.
  * It also records, per request, the flattened offset, the token count and whether the
  * flattening is well formed (1 <= Q_r <= K + 1 tokens inside [0, T_cap), token j carrying the

@@ -32,15 +32,14 @@ struct AttnPlanHeader {
 };
 
 // Cost model of the tensor-core kernel's work, in units of one 64-key cache page (about 0.75 us
-// of a CTA's time at full clock).  A segment's verify tokens and its query rows cost 5, a piece
-// (its epilogue, about 4 us, and the refill of the pipeline for the next piece) 10, merging the
-// partials of a split segment 8: the middle of the plateau of a sweep of the three constants,
-// timed on workloads of 64 to 1024 requests (the per-CTA finish times of one call put a piece
-// near 9 pages).  The head piece of a split segment usually merges, as the next CTA finishes the
-// segment's rest first.
-constexpr float kCostNewTile = 5.0f;
-constexpr float kCostPiece = 10.0f;
-constexpr float kCostMerge = 8.0f;
+// of a CTA's time at full clock).  A segment's verify tokens and its query rows cost 4, a piece
+// (its epilogue and the refill of the pipeline for the next piece) 7, merging the partials of a
+// split segment 6: the best of a sweep of the three constants, timed on workloads of 64 to 1024
+// requests; the plateau is flat to about 1%.  The head piece of a split segment usually merges,
+// as the next CTA finishes the segment's rest first.
+constexpr float kCostNewTile = 4.0f;
+constexpr float kCostPiece = 7.0f;
+constexpr float kCostMerge = 6.0f;
 // Candidate cost bounds the plan tests at once (one per thread of its single CTA).
 constexpr int kPlanCandidates = 1024;
 // Requests whose segment costs the plan keeps in shared memory (more go to the workspace).
@@ -60,6 +59,7 @@ struct AttnWs {
   int *cta_begin;    // [max_ctas + 1]: first unit of tensor-core CTA c; [tc_ctas] = total
   float *partials;   // [2 * max_ctas][rows_max][part_stride(D)]: acc[D], m, l per row
   float *seg_cost;   // [R]: modelled cost of a whole segment of request r (plan scratch)
+  int4 *cta_req;     // [max_ctas]: the request record of tensor-core CTA c's first segment
 };
 
 __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, int D,
@@ -74,6 +74,7 @@ __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, i
   const size_t o_par = off;
   off += align256((size_t)2 * max_ctas * rows_max * part_stride(D) * sizeof(float));
   const size_t o_sc = off;                 off += align256((size_t)R * sizeof(float));
+  const size_t o_crq = off;                off += align256((size_t)max_ctas * sizeof(int4));
   if (ws) {
     char *b = static_cast<char *>(base);
     ws->hdr = reinterpret_cast<AttnPlanHeader *>(b + o_hdr);
@@ -84,6 +85,7 @@ __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, i
     ws->cta_begin = reinterpret_cast<int *>(b + o_beg);
     ws->partials = reinterpret_cast<float *>(b + o_par);
     ws->seg_cost = reinterpret_cast<float *>(b + o_sc);
+    ws->cta_req = reinterpret_cast<int4 *>(b + o_crq);
   }
   return off;
 }
@@ -269,15 +271,18 @@ attn_plan_kernel(const int32_t *__restrict__ kv_len, const int32_t *__restrict__
     ws.hdr->tc_bound = bound;
   }
   __syncthreads();
+  // (the request records written above are visible to the whole block since its barriers)
   for (int c = tid; c < tc_ctas; c += blockDim.x) {
-    int4 st = make_int4(-1, 0, 0, 0);
+    int4 st = make_int4(-1, 0, 0, 0), rq = make_int4(0, 0, 0, 0);
     const int u0 = ws.cta_begin[c];
     if (u0 < ws.cta_begin[c + 1]) {
       int r, g, tiles, s0;
       find_segment(ws.tile_prefix, R, Hkv, u0, r, g, tiles, s0);
       st = make_int4(r, g, s0, tiles);
+      rq = ws.req[r];
     }
     ws.cta_start[c] = st;
+    ws.cta_req[c] = rq;  // with the start record, so a CTA's first piece needs no dependent load
   }
   if (tid == 0) {
     ws.hdr->R = R;

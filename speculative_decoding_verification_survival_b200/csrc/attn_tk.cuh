@@ -124,10 +124,9 @@ struct Meta {
   int t0, Q, n, rows, npages, ncache, ntiles, npass;  // npages: cache pages of the piece
   bool valid, last, newtile;                          // ncache: their 128-key tiles
 };
-__device__ __forceinline__ Meta piece_meta(const AttnArgs &a, int r, int ta, int tb, int tiles,
-                                           bool raise) {
+__device__ __forceinline__ Meta piece_meta(const AttnArgs &a, const int4 &rec, int ta, int tb,
+                                           int tiles, bool raise) {
   Meta m;
-  const int4 rec = __ldg(a.ws.req + r);
   m.t0 = rec.x;
   m.Q = rec.y;
   m.n = rec.z;
@@ -152,16 +151,27 @@ struct PieceIter {
   int u, u1;
   Ranges rg;
   int r, g, tiles, s0;  // current segment
+  int4 first_rec;       // the first segment's request record, from the plan's start records
+  bool have_first;
   __device__ __forceinline__ void init(const AttnArgs &a) {
+    // every load of the start issued at once (all in bounds for any grid up to the plan's
+    // maximum), so the first piece is one round trip away
     const int total = __ldg(&a.ws.hdr->total);
     const int ctas = __ldg(&a.ws.hdr->tc_ctas);
+    const int4 st = __ldg(a.ws.cta_start + blockIdx.x);
+    const int b0 = __ldg(a.ws.cta_begin + blockIdx.x), b1 = __ldg(a.ws.cta_begin + blockIdx.x + 1);
+    first_rec = __ldg(a.ws.cta_req + blockIdx.x);
+    have_first = false;
     if (ctas == (int)gridDim.x) {  // the plan's cost-balanced ranges
       rg.begin = a.ws.cta_begin;
       rg.W = 0;
       rg.ctas = ctas;
       rg.total = total;
-      const int4 st = __ldg(a.ws.cta_start + blockIdx.x);
       r = st.x; g = st.y; s0 = st.z; tiles = st.w;
+      u = b0;
+      u1 = (r < 0) ? u : min(b1, total);
+      have_first = true;
+      return;
     } else {  // a grid the plan did not prepare for: equal ranges, search the first segment
       rg.begin = nullptr;
       rg.W = (total + gridDim.x - 1) / gridDim.x;
@@ -206,7 +216,9 @@ struct PassIter {
   __device__ __forceinline__ bool first(const AttnArgs &a, Pass &p, bool raise) {
     if (!it.next(a, p.r, p.g, p.ta, p.tb, p.tiles, p.s0)) return false;
     p.h = 0;
-    p.m = piece_meta(a, p.r, p.ta, p.tb, p.tiles, raise);
+    const int4 rec = it.have_first ? it.first_rec : __ldg(a.ws.req + p.r);
+    it.have_first = false;
+    p.m = piece_meta(a, rec, p.ta, p.tb, p.tiles, raise);
     return true;
   }
   __device__ __forceinline__ bool next(const AttnArgs &a, const Pass &cur, Pass &p, bool raise) {

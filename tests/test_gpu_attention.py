@@ -239,7 +239,7 @@ def test_full_workload_structured_keys_and_values(name):
 
 
 # ---- the plan's cost-balanced ranges ----------------------------------------------------------
-_COST_NEW, _COST_PIECE, _COST_MERGE, _SEG_TAIL = 5.0, 10.0, 8.0, 8
+_COST_NEW, _COST_PIECE, _COST_MERGE, _SEG_TAIL = 4.0, 7.0, 6.0, 8
 
 
 def _plan_ranges(step, cfg):
