@@ -42,8 +42,9 @@ constexpr float kCostPiece = 7.0f;
 constexpr float kCostMerge = 6.0f;
 // Candidate cost bounds the plan tests at once (one per thread of its single CTA).
 constexpr int kPlanCandidates = 1024;
-// Requests whose segment costs the plan keeps in shared memory (more go to the workspace).
-constexpr int kPlanSmemRequests = 8192;
+// Requests whose unit prefix the plan keeps in shared memory for the candidate fills (more are
+// read from the workspace).
+constexpr int kPlanSmemRequests = 4096;
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -59,7 +60,9 @@ struct AttnWs {
   int *cta_begin;    // [max_ctas + 1]: first unit of tensor-core CTA c; [tc_ctas] = total
   float *partials;   // [2 * max_ctas][rows_max][part_stride(D)]: acc[D], m, l per row
   float *seg_cost;   // [R]: modelled cost of a whole segment of request r (plan scratch)
+  int *seg_c;        // [R]: the same as an integer (plan scratch past kPlanSmemRequests)
   int4 *cta_req;     // [max_ctas]: the request record of tensor-core CTA c's first segment
+  int *cand_begin;   // [kPlanCandidates][max_ctas + 1]: each candidate fill's range starts
 };
 
 __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, int D,
@@ -75,6 +78,9 @@ __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, i
   off += align256((size_t)2 * max_ctas * rows_max * part_stride(D) * sizeof(float));
   const size_t o_sc = off;                 off += align256((size_t)R * sizeof(float));
   const size_t o_crq = off;                off += align256((size_t)max_ctas * sizeof(int4));
+  const size_t o_sgc = off;                off += align256((size_t)R * sizeof(int));
+  const size_t o_cbg = off;
+  off += align256((size_t)kPlanCandidates * (max_ctas + 1) * sizeof(int));
   if (ws) {
     char *b = static_cast<char *>(base);
     ws->hdr = reinterpret_cast<AttnPlanHeader *>(b + o_hdr);
@@ -86,6 +92,8 @@ __host__ __device__ inline size_t attn_ws_layout(int R, int Hkv, int rows_max, i
     ws->partials = reinterpret_cast<float *>(b + o_par);
     ws->seg_cost = reinterpret_cast<float *>(b + o_sc);
     ws->cta_req = reinterpret_cast<int4 *>(b + o_crq);
+    ws->cand_begin = reinterpret_cast<int *>(b + o_cbg);
+    ws->seg_c = reinterpret_cast<int *>(b + o_sgc);
   }
   return off;
 }
@@ -115,9 +123,10 @@ __device__ __forceinline__ void find_segment(const int *__restrict__ tile_prefix
 // Greedy fill of CTAs in unit order under a cost bound: a segment goes whole into the current
 // CTA if it fits; otherwise the CTA takes a head piece of an even number of cache pages (at
 // least 2, with the piece and merge costs) and the rest continues in the next CTAs (which may
-// cut it again); a bound under which not even a two-page piece fits counts as infeasible.  A range boundary never falls inside a segment's verify-token units.  Returns
-// the number of CTAs used (stops counting past `cap`); when `begin` is given, records the first
-// unit of every CTA used (begin[0] = 0).
+// cut it again); a bound under which not even a two-page piece fits counts as infeasible.  A
+// range boundary never falls inside a segment's verify-token units.  Returns the number of CTAs
+// used (stops counting past `cap`); when `begin` is given, records the first unit of every CTA
+// used (begin[0] = 0).
 __device__ int plan_fill(const int *__restrict__ tile_prefix, const float *seg_cost, int R, int Hkv,
                          float bound, int cap, int *begin) {
   int used = 1;
@@ -151,6 +160,72 @@ __device__ int plan_fill(const int *__restrict__ tile_prefix, const float *seg_c
         if (mid < 2) return cap + 1;  // not even a two-page piece fits: the bound is infeasible
         done = min(u, done + mid);
       }
+    }
+  }
+  return used;
+}
+
+// The same greedy fill, jumping over the whole segments that fit.  The costs are integers and a
+// whole segment of request r costs its units plus kNew + kPiece - kSegTail, so the cost of all
+// segments of the requests before r is pq(r) = tile_prefix[r] + r * Hkv * (kNew + kPiece -
+// kSegTail): the run of whole segments that fits in a CTA's remaining capacity is found by a
+// binary search on it, and only the segments that are cut take the steps above.  A fill costs
+// O(CTAs * log R) instead of O(R * Hkv), with the same ranges as plan_fill for the same bound.
+// The caller checks that pq(R) fits an int.
+__device__ int plan_fill_jump(const int *tile_prefix, const int *segc, int R, int Hkv,
+                              float bound, int cap, int *begin) {
+  const int B = (int)floorf(bound);  // every cost is an integer: cost <= bound <=> cost <= B
+  constexpr int kNew = (int)kCostNewTile, kPiece = (int)kCostPiece, kMerge = (int)kCostMerge;
+  const int step = Hkv * (kNew + kPiece - kSegTail);
+  auto pq = [&](int r) { return tile_prefix[r] + r * step; };
+  int used = 1, cur = 0;
+  if (begin) begin[0] = 0;
+  int r = 0, g = 0;  // the next segment
+  while (r < R && used <= cap) {
+    const int start = pq(r) + g * segc[r];
+    const int limit = start + (B - cur);  // the cost prefix this CTA can reach
+    // the last request whose start the CTA reaches: largest r2 in [r, R] with pq(r2) <= limit,
+    // by a galloping search from r (a CTA spans few requests), then bisection
+    int lo = r, stp = 1;
+    while (lo + stp <= R && pq(lo + stp) <= limit) {
+      lo += stp;
+      stp <<= 1;
+    }
+    int hi = min(R, lo + stp - 1);
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pq(mid) <= limit) lo = mid; else hi = mid - 1;
+    }
+    const int r2 = lo;
+    if (r2 == R) break;  // everything left fits
+    const int p2 = pq(r2), c2 = segc[r2];
+    // segments of r2 that fit whole: floor((limit - p2) / c2) by a float quotient and a fix-up
+    // (small integers, exact in float)
+    int g2 = (int)__fdividef((float)(limit - p2), (float)c2);
+    if ((g2 + 1) * c2 <= limit - p2) ++g2;
+    if (g2 * c2 > limit - p2) --g2;
+    g2 = min(Hkv - 1, g2);
+    cur += p2 + g2 * c2 - start;
+    r = r2;
+    g = g2;
+    // segment (r, g) does not fit whole: cut it
+    const int u = c2 - kNew - kPiece;  // cache pages of a segment
+    const int s0 = tile_prefix[r] + g * (u + kSegTail);
+    int done = 0;
+    const int head = (B - cur - kPiece - kMerge) & ~1;
+    if (head >= 2 && head < u) done = head;  // head piece in the current CTA
+    while (true) {
+      ++used;
+      if (begin && used <= cap) begin[used - 1] = s0 + done;
+      const int rest = (u - done) + kNew + kPiece;
+      if (rest <= B || used > cap) { cur = rest; break; }
+      const int midp = (B - kPiece - (done == 0 ? kMerge : 0)) & ~1;
+      if (midp < 2) return cap + 1;  // not even a two-page piece fits: the bound is infeasible
+      done = min(u, done + midp);
+    }
+    if (++g == Hkv) {
+      g = 0;
+      ++r;
     }
   }
   return used;
@@ -249,27 +324,53 @@ attn_plan_kernel(const int32_t *__restrict__ kv_len, const int32_t *__restrict__
   // starts.
   const float lo = s_tot / (float)tc_ctas;
   const float hi = lo + s_pmax[0] + kCostMerge + kCostPiece;
-  __shared__ float s_cost[kPlanSmemRequests];
+  // The fills read the unit prefix from shared memory when it fits; a cost total that does not
+  // fit an int (far beyond any real batch) falls back to the segment-by-segment float fill.
+  __shared__ int s_tp[kPlanSmemRequests + 1], s_c[kPlanSmemRequests];
   const bool staged = R <= kPlanSmemRequests;
-  float *cost = staged ? s_cost : ws.seg_cost;
-  for (int r = tid; r < R; r += blockDim.x)
-    cost[r] = (float)((ws.tile_prefix[r + 1] - ws.tile_prefix[r]) / Hkv - kSegTail) +
-              kCostNewTile + kCostPiece;
+  int *segc = staged ? s_c : ws.seg_c;
+  if (staged)
+    for (int r = tid; r <= R; r += blockDim.x) s_tp[r] = ws.tile_prefix[r];
+  for (int r = tid; r < R; r += blockDim.x)  // a whole segment's cost, per request
+    segc[r] = (ws.tile_prefix[r + 1] - ws.tile_prefix[r]) / Hkv - kSegTail + (int)kCostNewTile +
+              (int)kCostPiece;
+  const long long cost_total =
+      (long long)total + (long long)R * Hkv * (long long)(kCostNewTile + kCostPiece - kSegTail);
+  const bool jump = cost_total < (long long)INT_MAX / 2;
+  if (!jump)
+    for (int r = tid; r < R; r += blockDim.x)
+      ws.seg_cost[r] = (float)((ws.tile_prefix[r + 1] - ws.tile_prefix[r]) / Hkv - kSegTail) +
+                       kCostNewTile + kCostPiece;
   __syncthreads();
-  if (tid < kPlanCandidates) {
-    const float cand = lo + (hi - lo) * (float)(tid + 1) / (float)kPlanCandidates;
-    if (plan_fill(ws.tile_prefix, cost, R, Hkv, cand, tc_ctas, nullptr) <= tc_ctas)
-      atomicMin(&s_best, tid);
+  const int *tp = staged ? s_tp : ws.tile_prefix;
+  // Every cost is an integer, so bounds with the same integer part give the same fill: the
+  // candidates are integers from floor(lo) + 1 up, at a spacing that covers (lo, hi] with at
+  // most kPlanCandidates of them (the last one is hi or more: always feasible).  Small batches
+  // then test a few dozen bounds, not a thousand copies of them.
+  const int ilo = (int)floorf(lo);
+  const int span = max(1, (int)ceilf(hi) - ilo);
+  const int spacing = (span + kPlanCandidates - 1) / kPlanCandidates;
+  const int ncand = (span + spacing - 1) / spacing;
+  // Each fill records its range starts in a scratch row of its own; the winner's row is then
+  // copied, so no fill runs twice.
+  __shared__ int s_used[kPlanCandidates];
+  if (tid < ncand) {
+    const float cand = (float)(ilo + (tid + 1) * spacing);
+    int *mine = ws.cand_begin + (size_t)tid * (tc_ctas + 1);
+    const int need = jump ? plan_fill_jump(tp, segc, R, Hkv, cand, tc_ctas, mine)
+                          : plan_fill(ws.tile_prefix, ws.seg_cost, R, Hkv, cand, tc_ctas, mine);
+    s_used[tid] = need;
+    if (need <= tc_ctas) atomicMin(&s_best, tid);
   }
   __syncthreads();
-  const float bound = lo + (hi - lo) * (float)(min(s_best, kPlanCandidates - 1) + 1) /
-                               (float)kPlanCandidates;
-  if (tid == 0) {
-    const int used = plan_fill(ws.tile_prefix, cost, R, Hkv, bound, tc_ctas, ws.cta_begin);
-    // trailing CTAs get empty ranges; had no bound fitted, the last CTA would take the rest
-    for (int c = min(used, tc_ctas); c <= tc_ctas; ++c) ws.cta_begin[c] = total;
-    ws.hdr->tc_bound = bound;
-  }
+  const int best = min(s_best, ncand - 1);
+  const float bound = (float)(ilo + (best + 1) * spacing);
+  const int used = min(s_used[best], tc_ctas);
+  const int *win = ws.cand_begin + (size_t)best * (tc_ctas + 1);
+  // the winner's starts; trailing CTAs get empty ranges (had no bound fitted, the last CTA would
+  // take the rest)
+  for (int c = tid; c <= tc_ctas; c += blockDim.x) ws.cta_begin[c] = c < used ? win[c] : total;
+  if (tid == 0) ws.hdr->tc_bound = bound;
   __syncthreads();
   // (the request records written above are visible to the whole block since its barriers)
   for (int c = tid; c < tc_ctas; c += blockDim.x) {
