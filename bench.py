@@ -129,13 +129,13 @@ class ClockSampler:
 # any change to those voids the figure.  Entries: (sha, bytes, algorithmic bytes of the capture);
 # a capture of another size of the same workload is scaled by algorithmic bytes.
 NCU_TRAFFIC = {
-    # one launch of the full workload (a 1-pass capture): 22 408 662 528 B read + 37 221 632 B
+    # one launch of the full workload (a 1-pass capture): 22 409 124 864 B read + 38 480 384 B
     # written, 22 324 592 640 algorithmic bytes
-    "lognormal-1024req": ("9ccca0085399ec954df78b80b3b3a56acba7926a", 22445884160, 22324592640),
-    "lognormal-1024req-greedy": ("9ccca0085399ec954df78b80b3b3a56acba7926a", 22445884160,
+    "lognormal-1024req": ("79531114a27673b7ae189c6abc443ed3527d8362", 22447605248, 22324592640),
+    "lognormal-1024req-greedy": ("79531114a27673b7ae189c6abc443ed3527d8362", 22447605248,
                                  22324592640),
-    # 626 938 112 B read + 4 952 064 B written, 621 088 768 algorithmic bytes
-    "qwen3-4b-64req": ("9ccca0085399ec954df78b80b3b3a56acba7926a", 631890176, 621088768),
+    # 627 339 264 B read + 5 733 376 B written, 621 088 768 algorithmic bytes
+    "qwen3-4b-64req": ("79531114a27673b7ae189c6abc443ed3527d8362", 633072640, 621088768),
 }
 
 ATTN_SOURCES = ("attn_tk.cuh", "attn_common.cuh", "ptx_sm100.cuh", "common.cuh", "dspark.cu")
