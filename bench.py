@@ -103,7 +103,7 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
+        sm, mx, pw, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -114,12 +114,17 @@ class ClockSampler:
                 mx.append(float(parts[1]))
             except ValueError:
                 continue
+            try:
+                pw.append(float(parts[2]))
+            except ValueError:
+                pass
             for nm, v in zip(names, parts[4:8]):
                 if v.lower() == "active":
                     reasons.add(nm)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "power_w": statistics.median(pw) if pw else None,
                 "reasons": sorted(reasons), "samples": len(sm),
                 "sufficient": len(sm) >= MIN_CLOCK_SAMPLES}
 
@@ -129,13 +134,13 @@ class ClockSampler:
 # any change to those voids the figure.  Entries: (sha, bytes, algorithmic bytes of the capture);
 # a capture of another size of the same workload is scaled by algorithmic bytes.
 NCU_TRAFFIC = {
-    # one launch of the full workload (a 1-pass capture): 22 409 124 864 B read + 38 480 384 B
+    # one launch of the full workload (a 1-pass capture): 22 411 018 496 B read + 37 052 416 B
     # written, 22 324 592 640 algorithmic bytes
-    "lognormal-1024req": ("79531114a27673b7ae189c6abc443ed3527d8362", 22447605248, 22324592640),
-    "lognormal-1024req-greedy": ("79531114a27673b7ae189c6abc443ed3527d8362", 22447605248,
+    "lognormal-1024req": ("6c751188c09a7f55360fe03ab670a01ae474a9aa", 22448070912, 22324592640),
+    "lognormal-1024req-greedy": ("6c751188c09a7f55360fe03ab670a01ae474a9aa", 22448070912,
                                  22324592640),
-    # 627 339 264 B read + 5 733 376 B written, 621 088 768 algorithmic bytes
-    "qwen3-4b-64req": ("79531114a27673b7ae189c6abc443ed3527d8362", 633072640, 621088768),
+    # 626 557 696 B read + 4 208 128 B written, 621 088 768 algorithmic bytes
+    "qwen3-4b-64req": ("6c751188c09a7f55360fe03ab670a01ae474a9aa", 630765824, 621088768),
 }
 
 ATTN_SOURCES = ("attn_tk.cuh", "attn_common.cuh", "ptx_sm100.cuh", "common.cuh", "dspark.cu")

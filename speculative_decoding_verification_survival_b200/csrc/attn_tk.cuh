@@ -18,18 +18,22 @@
 // segment with 33..64 rows is taken in two passes of 32 rows over the same keys (each pass
 // reads its keys again; the schedules of the benchmark workloads give at most 32 rows).
 //
-// Per CTA (384 threads, 12 warps): warp 8 loads K (TMA, one 128-byte-swizzled 4-D box per
-// page, a ring of 3 tiles with one barrier each), warp 10 loads V (the same, its own ring), one
-// thread of warp 9 issues the S^T MMAs and one of warp 11 the P.V MMAs, warps 0-7 do the softmax
-// and the epilogue: warp w reads the lanes of its
+// Per CTA (512 threads, 16 warps): warps 8 and 12 load K (TMA, one 128-byte-swizzled 4-D box per
+// page, page 0 and page 1 of every tile, a ring of 3 tiles with one barrier each), warps 10 and
+// 14 load V (the same, its own ring): one warp issues about one box per 850 cycles, and two per
+// ring keep up with HBM also at a power-capped clock.  One thread of warp 9 issues the S^T MMAs
+// and one of warp 11 the P.V MMAs; warps 13 and 15 idle.  Warpgroups 2 and 3 hand registers to
+// warpgroups 0 and 1 (setmaxnreg: 88 and 168 per thread, from 128 at launch), which do the
+// softmax and the epilogue: warp w reads the lanes of its
 // quadrant q = w % 4 (keys 32q .. 32q + 31 of the tile, and d = 32q .. 32q + 31 of O^T) and the
 // columns of its half hf = w / 4 of the rows, so every thread holds one key's scores for 16
 // rows.  A row's reference maximum comes from the pass's first tile and is raised only when a
 // score exceeds it by more than 2^8 (log2 domain): the 128 threads of a half vote every tile and
 // a tile that exceeds takes the slow path (row maxima by warp shuffles and a shared-memory
 // exchange, tensor-memory rescale of O^T).  Row sums stay per thread (per key) until the pass's
-// epilogue.  Every mbarrier wait is bounded (ptx::mbar_wait); on timeout the CTA records
-// DSPARK_DERR_TIMEOUT, skips the remaining work and still releases its TMEM.
+// epilogue.  Every mbarrier wait is bounded (ptx::mbar_wait, its polling loop out of line in the
+// MMA issuers, inlined elsewhere); on timeout the CTA records DSPARK_DERR_TIMEOUT, skips the
+// remaining work and still releases its TMEM.
 #pragma once
 
 #include "attn_generic.cuh"
@@ -45,9 +49,16 @@ constexpr int kMaxPairs = 4;
 static_assert(kPairsK <= kMaxPairs && kPairsV <= kMaxPairs && 8 * kMaxPairs <= 48, "slot counts");
 constexpr int kSoftmaxWarps = 8;
 constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+// warpgroup 2: K producer (page 0 of each tile), S^T issuer, V producer (page 0), P.V issuer;
+// warpgroup 3: K producer (page 1), idle, V producer (page 1), idle
 constexpr int kWarpK = kSoftmaxWarps, kWarpMma = kSoftmaxWarps + 1, kWarpV = kSoftmaxWarps + 2,
-              kWarpPV = kSoftmaxWarps + 3;
-constexpr int kThreads = kSoftmaxThreads + 128;
+              kWarpPV = kSoftmaxWarps + 3, kWarpK2 = kSoftmaxWarps + 4, kWarpV2 = kSoftmaxWarps + 6;
+constexpr int kThreads = kSoftmaxThreads + 256;
+// registers per thread: at launch (the pool: 65536 / 512), then the softmax warpgroups and the
+// others after the split; the shares add up to the pool
+constexpr int kRegsLaunch = 128, kRegsSoftmax = 168, kRegsOther = 88;
+static_assert(kRegsSoftmax * kSoftmaxThreads + kRegsOther * (kThreads - kSoftmaxThreads) <=
+                  kRegsLaunch * kThreads, "register split");
 constexpr int kD = 128;
 constexpr int kNewRows = 16;                         // verify tokens per tile (K + 1 <= 16)
 constexpr int kN = 32;                               // query rows per pass (the MMAs' N)
@@ -316,7 +327,7 @@ __device__ __forceinline__ void softmax_tile(const AttnArgs &a, float (&mref)[kR
     // previous tile's P.V has completed
     const bool rescale_o = !first_tile;
     if (rescale_o) {
-      ptx::mbar_wait(aux + kBarODone, (gt - 1) & 1, abort_flag);
+      ptx::mbar_wait_inl(aux + kBarODone, (gt - 1) & 1, abort_flag);
       ptx::tc_fence_after();
     }
     const uint32_t o_taddr = tmem + lane_base + kColO + hf * kRH;
@@ -363,7 +374,7 @@ __device__ __forceinline__ void softmax_tile(const AttnArgs &a, float (&mref)[kR
   }
   // the single P^T buffer was last read by the P.V of tile gt - 1
   if (gt >= 1) {
-    ptx::mbar_wait(aux + kBarODone, (gt - 1) & 1, abort_flag);
+    ptx::mbar_wait_inl(aux + kBarODone, (gt - 1) & 1, abort_flag);
     ptx::tc_fence_after();
   }
   // P^T row of key kk (MN-major, 64-byte swizzle): rows hf*16 .. hf*16 + 15 = chunks 2hf, 2hf+1
@@ -396,12 +407,13 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
   auto bar = [&](uint32_t off, int i) { return aux + off + 8u * (uint32_t)i; };
 
   if (tid == 0) {
+    // a tile's full barrier: one arrival (with its transaction bytes) per page producer
     for (int i = 0; i < kPairsK; ++i) {
-      ptx::mbar_init(bar(kBarKFull, i), 1);
+      ptx::mbar_init(bar(kBarKFull, i), 2);
       ptx::mbar_init(bar(kBarKEmpty, i), 1);
     }
     for (int i = 0; i < kPairsV; ++i) {
-      ptx::mbar_init(bar(kBarVFull, i), 1);
+      ptx::mbar_init(bar(kBarVFull, i), 2);
       ptx::mbar_init(bar(kBarVEmpty, i), 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -437,186 +449,185 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
   // launch may then start its own prologue as soon as SMs free up.
   ptx::grid_dependency_wait();
   ptx::grid_launch_dependents();
-
-  if (warp == kWarpK || warp == kWarpV) {
-    // ------------------------------------------------------------------ TMA producers
-    // One warp loads K, another V, a tile (two pages) per ring slot: one barrier and one
-    // transaction count per tile, one 4-D box per page.  The whole warp walks the tiles; lane 0
-    // waits on the barriers and issues the copies.  The block-table entries come 32 at a time,
-    // lane i holding entry base + i, and the chunk after the current one is loaded ahead, so a
-    // page's lookup is a register shuffle and no copy waits on a dependent global load.  Tile gt
-    // uses tile slot gt mod 3 of its ring.
-    const bool is_k = (warp == kWarpK);
-    const uint32_t full0 = is_k ? kBarKFull : kBarVFull, empty0 = is_k ? kBarKEmpty : kBarVEmpty;
-    const int v = is_k ? 0 : 1;
-    const CUtensorMap *nmap = is_k ? &tmap_kn : &tmap_vn;
-    const int npairs = is_k ? kPairsK : kPairsV;
-    // every cached page is read once per pass by one CTA: let it leave L2 first, so that the
-    // split-KV partials written early in the kernel are still there when they are merged
-    const uint64_t stream_policy = ptx::l2_policy_evict_first();
-    int last_use[kMaxPairs];  // latest slot use that was armed, -1 if none
+  if (warp >= kSoftmaxWarps) {
+    // producers and issuers (warpgroups 2 and 3) hand registers to the softmax warpgroups
+    ptx::setmaxnreg_dec<kRegsOther>();
+    if (warp == kWarpK || warp == kWarpV || warp == kWarpK2 || warp == kWarpV2) {
+      // ------------------------------------------------------------------ TMA producers
+      // Two warps load K and two V, a tile (two pages) per ring slot and one barrier per tile:
+      // producer hp of a ring loads page hp of every tile as one 4-D box (a warp issues about one
+      // box per 850 cycles, so two per ring keep up with HBM at a power-capped clock) and arrives
+      // with its bytes.  The whole warp walks the tiles; lane 0 waits on the barriers and issues
+      // the copies.  The block-table entries come 32 at a time,
+      // lane i holding entry base + i, and the chunk after the current one is loaded ahead, so a
+      // page's lookup is a register shuffle and no copy waits on a dependent global load.  Tile gt
+      // uses tile slot gt mod 3 of its ring.
+      const bool is_k = (warp == kWarpK || warp == kWarpK2);
+      const int hp = (warp == kWarpK2 || warp == kWarpV2) ? 1 : 0;  // the page of the tile
+      const uint32_t full0 = is_k ? kBarKFull : kBarVFull, empty0 = is_k ? kBarKEmpty : kBarVEmpty;
+      const int v = is_k ? 0 : 1;
+      const CUtensorMap *nmap = is_k ? &tmap_kn : &tmap_vn;
+      const int npairs = is_k ? kPairsK : kPairsV;
+      // every cached page is read once per pass by one CTA: let it leave L2 first, so that the
+      // split-KV partials written early in the kernel are still there when they are merged
+      const uint64_t stream_policy = ptx::l2_policy_evict_first();
+      int last_use[kMaxPairs];  // latest slot use that was armed, -1 if none
 #pragma unroll
-    for (int k = 0; k < kMaxPairs; ++k) last_use[k] = -1;
-    auto bt_chunk = [&](int rr, int b0) -> int {
-      const int i = b0 + lane;
-      return (i < a.max_pages) ? __ldg(a.block_table + (size_t)rr * a.max_pages + i) : -1;
-    };
-    int creq = -1, cbase = 0, cval = -1, nbase = 0, nval = -1;
-    // the page behind block-table index bi of request rr (a warp-wide call)
-    auto page_of = [&](int rr, int bi) -> int {
-      if (rr != creq || bi < cbase || bi >= cbase + 32) {
-        if (rr == creq && bi >= nbase && bi < nbase + 32) {
-          cbase = nbase;
-          cval = nval;
-        } else {
-          cbase = bi;
-          cval = bt_chunk(rr, cbase);
+      for (int k = 0; k < kMaxPairs; ++k) last_use[k] = -1;
+      auto bt_chunk = [&](int rr, int b0) -> int {
+        const int i = b0 + lane;
+        return (i < a.max_pages) ? __ldg(a.block_table + (size_t)rr * a.max_pages + i) : -1;
+      };
+      int creq = -1, cbase = 0, cval = -1, nbase = 0, nval = -1;
+      // the page behind block-table index bi of request rr (a warp-wide call)
+      auto page_of = [&](int rr, int bi) -> int {
+        if (rr != creq || bi < cbase || bi >= cbase + 32) {
+          if (rr == creq && bi >= nbase && bi < nbase + 32) {
+            cbase = nbase;
+            cval = nval;
+          } else {
+            cbase = bi;
+            cval = bt_chunk(rr, cbase);
+          }
+          creq = rr;
+          nbase = cbase + 32;
+          nval = bt_chunk(rr, nbase);  // the next chunk, ahead of its use
         }
-        creq = rr;
-        nbase = cbase + 32;
-        nval = bt_chunk(rr, nbase);  // the next chunk, ahead of its use
-      }
-      return __shfl_sync(0xffffffffu, cval, bi - cbase);
-    };
-    TileCursor tc;
-    tc.init(a);
-    while (__shfl_sync(0xffffffffu, (tc.ok && !*abort_flag) ? 1 : 0, 0)) {
-      const Meta &m = tc.p.m;
-      const uint32_t slot = tc.gt % npairs;
-      if (lane == 0) ptx::mbar_wait(bar(empty0, slot), ((tc.gt / npairs) & 1) ^ 1, abort_flag);
-      if (__shfl_sync(0xffffffffu, *abort_flag, 0) != 0) break;
-      const uint32_t fb = bar(full0, slot), dst = ring(v, slot);
-      if (tc.j < m.ncache) {
-        const int npg = min(2, m.npages - 2 * tc.j);  // pages of the piece in this tile
-        int pages[2];
-        int key0[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          key0[h] = (tc.p.ta + 2 * tc.j + h) * kPage;
-          pages[h] = (h < npg) ? page_of(tc.p.r, key0[h] / a.page_size) : -1;
-        }
-        if (lane == 0) {
-          ptx::mbar_arrive_expect_tx(fb, (uint32_t)npg * kPageBytes);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (h < npg) {
+        return __shfl_sync(0xffffffffu, cval, bi - cbase);
+      };
+      TileCursor tc;
+      tc.init(a);
+      while (__shfl_sync(0xffffffffu, (tc.ok && !*abort_flag) ? 1 : 0, 0)) {
+        const Meta &m = tc.p.m;
+        const uint32_t slot = tc.gt % npairs;
+        if (lane == 0) ptx::mbar_wait_inl(bar(empty0, slot), ((tc.gt / npairs) & 1) ^ 1, abort_flag);
+        if (__shfl_sync(0xffffffffu, *abort_flag, 0) != 0) break;
+        const uint32_t fb = bar(full0, slot), dst = ring(v, slot);
+        if (tc.j < m.ncache) {
+          const bool has = hp < min(2, m.npages - 2 * tc.j);  // the piece has this page
+          const int key0 = (tc.p.ta + 2 * tc.j + hp) * kPage;
+          const int page = has ? page_of(tc.p.r, key0 / a.page_size) : -1;
+          if (lane == 0) {
+            if (has) {
+              ptx::mbar_arrive_expect_tx(fb, kPageBytes);
               int row = oob_row;
-              const int page = pages[h];
               if (page >= 0 && page < a.num_pages) {
-                row = ((page * 2 + v) * a.Hkv + tc.p.g) * a.page_size + key0[h] % a.page_size;
+                row = ((page * 2 + v) * a.Hkv + tc.p.g) * a.page_size + key0 % a.page_size;
               } else if (is_k) {
                 raise_error(DSPARK_DERR_PAGE);
               }
-              ptx::tma_load_4d_hint(dst + h * kPageBytes, &tmap_kv, fb, 0, 0, 0, row >> 3,
+              ptx::tma_load_4d_hint(dst + hp * kPageBytes, &tmap_kv, fb, 0, 0, 0, row >> 3,
                                     stream_policy);
+            } else {
+              ptx::mbar_arrive(fb);
             }
           }
-        }
-      } else {  // the verify tokens: 16 rows of KV head g, two boxes of 8 tokens
-        if (lane == 0) {
-          ptx::mbar_arrive_expect_tx(fb, kNewBytes);
-          ptx::tma_load_4d(dst, nmap, fb, 0, m.t0, 0, tc.p.g);
-          ptx::tma_load_4d(dst + kGroupBytes, nmap, fb, 0, m.t0 + 8, 0, tc.p.g);
-        }
-      }
-      last_use[slot] = (int)tc.gt;
-      tc.advance(a);
-    }
-    // never leave the CTA with a bulk copy in flight: wait for the latest armed use of every
-    // slot (its phase is the newest one the slot's barrier can complete)
-    if (lane == 0) {
-      volatile int no_abort = 0;
-      for (int k = 0; k < npairs; ++k)
-        if (last_use[k] >= 0)
-          ptx::mbar_wait(bar(full0, k), ((uint32_t)last_use[k] / npairs) & 1, &no_abort);
-    }
-  } else if (warp == kWarpMma || warp == kWarpPV) {
-    // ------------------------------------------------------------------ MMA issuers
-    // One thread issues the S^T MMAs (warp 9), another the P.V MMAs (warp 11): each walks the
-    // tiles in order and waits (bounded) on its own barriers, and the two overlap the per-issue
-    // work that surrounds the MMAs.  They touch disjoint tensor memory (S^T buffers, O^T) and
-    // shared memory (K ring and query rows, V ring and P^T); P.V(j) needs P^T(j), which the
-    // softmax warps publish only after loading S^T(j).  S^T(j) overwrites the buffer of
-    // S^T(j - 2), which the softmax warps release as soon as they have loaded it, so S^T(j + 2)
-    // can go out while the softmax of tile j runs.
-    if (lane == 0) {
-      const bool is_s = (warp == kWarpMma);
-      TileCursor c;
-      c.init(a);
-      // P^T as B: MN-major with 64-byte swizzle, 8 keys per 512-byte atom
-      const uint64_t bd_p = ptx::smem_desc_sw64(pbase, 16, 512);
-      uint32_t issued = 0;
-      for (; c.ok; c.advance(a)) {
-        if (is_s) {
-          const uint32_t pair = c.gt % kPairsK, ph = (c.gt / kPairsK) & 1;
-          const int qb = c.pq & 1;
-          if (c.gt >= 2) ptx::mbar_wait(bar(kBarSFree, c.gt & 1), ((c.gt - 2) >> 1) & 1, abort_flag);
-          if (c.j == 0) ptx::mbar_wait(bar(kBarQFull, qb), (c.pq >> 1) & 1, abort_flag);
-          ptx::mbar_wait(bar(kBarKFull, pair), ph, abort_flag);
-          if (*abort_flag) break;
-          ptx::tc_fence_after();
-          const uint32_t d_tmem = tmem + kColS + (c.gt & 1) * kN;
-          // K tile as A (K-major: the keys on the lanes, groups of 8 keys 2048 bytes apart),
-          // the rows as B (K-major); 16 d per k-step: 32 bytes within the 128-byte atom rows,
-          // the d-halves 1024 bytes apart
-          const uint64_t a0 = ptx::smem_desc_sw128(ring(0, pair), 16, kGroupBytes);
-          const uint64_t a1 = ptx::smem_desc_sw128(ring(0, pair) + 1024, 16, kGroupBytes);
-          const uint64_t b0 = ptx::smem_desc_sw128(qbuf(qb, 0), 16, 1024);
-          const uint64_t b1 = ptx::smem_desc_sw128(qbuf(qb, 1), 16, 1024);
-#pragma unroll
-          for (int k = 0; k < kD / 16; ++k) {
-            const uint64_t off = (uint64_t)((k & 3) * 2);
-            ptx::mma_bf16_ss(d_tmem, (k < 4 ? a0 : a1) + off, (k < 4 ? b0 : b1) + off, kIdescS,
-                             k > 0 ? 1u : 0u);
+        } else {  // the verify tokens: 16 rows of KV head g, a box of 8 tokens per producer
+          if (lane == 0) {
+            ptx::mbar_arrive_expect_tx(fb, kNewBytes / 2);
+            ptx::tma_load_4d(dst + hp * kGroupBytes, nmap, fb, 0, m.t0 + 8 * hp, 0, tc.p.g);
           }
-          ptx::mma_commit(bar(kBarSFull, c.gt & 1));
-          ptx::mma_commit(bar(kBarKEmpty, pair));
-          // the pass's last S^T read of its rows: the buffer may be refilled
-          if (c.j == c.p.m.ntiles - 1) ptx::mma_commit(bar(kBarQEmpty, qb));
-        } else {
-          const uint32_t pair = c.gt % kPairsV, ph = (c.gt / kPairsV) & 1;
-          if (c.j == 0) ptx::mbar_wait(bar(kBarOFree, 0), (c.pq & 1) ^ 1, abort_flag);
-          ptx::mbar_wait(bar(kBarPFull, 0), c.gt & 1, abort_flag);
-          ptx::mbar_wait(bar(kBarVFull, pair), ph, abort_flag);
-          if (*abort_flag) break;
-          ptx::tc_fence_after();
-          const Meta &m = c.p.m;
-          const int jj = c.j;
-          const int ksteps = (jj < m.ncache) ? (min(kTK, m.npages * kPage - jj * kTK) / 16)
-                                             : kNewRows / 16;
-          // V^T as A: MN-major (D on the lanes, d-halves 1024 bytes apart, groups of 8 keys
-          // 2048 apart); fully unrolled k-steps with compile-time descriptor offsets (16 keys:
-          // 4096 bytes of V, 1024 of P^T)
-          const uint64_t ad0 = ptx::smem_desc_sw128(ring(1, pair), 1024, kGroupBytes);
-          const uint32_t acc0 = jj > 0 ? 1u : 0u;
-          if (ksteps == kTK / 16) {
-#pragma unroll
-            for (int k = 0; k < kTK / 16; ++k)
-              ptx::mma_bf16_ss(tmem + kColO, ad0 + (uint64_t)(k * 256), bd_p + (uint64_t)(k * 64),
-                               kIdescPV, k > 0 ? 1u : acc0);
-          } else if (ksteps == kPage / 16) {
-#pragma unroll
-            for (int k = 0; k < kPage / 16; ++k)
-              ptx::mma_bf16_ss(tmem + kColO, ad0 + (uint64_t)(k * 256), bd_p + (uint64_t)(k * 64),
-                               kIdescPV, k > 0 ? 1u : acc0);
-          } else {
-            ptx::mma_bf16_ss(tmem + kColO, ad0, bd_p, kIdescPV, acc0);
-          }
-          ptx::mma_commit(bar(kBarODone, 0));
-          ptx::mma_commit(bar(kBarVEmpty, pair));
         }
-        ++issued;
+        last_use[slot] = (int)tc.gt;
+        tc.advance(a);
       }
-      // every MMA this thread issued has completed before the CTA releases shared memory and
-      // TMEM, also after an abort (each issuer drains through its own barrier)
-      if (issued > 0) {
-        const uint32_t drain = bar(kBarDrain, is_s ? 0 : 1);
-        ptx::mma_commit(drain);
+      // never leave the CTA with a bulk copy in flight: wait for the latest armed use of every
+      // slot (its phase is the newest one the slot's barrier can complete)
+      if (lane == 0) {
         volatile int no_abort = 0;
-        ptx::mbar_wait(drain, 0, &no_abort);
+        for (int k = 0; k < npairs; ++k)
+          if (last_use[k] >= 0)
+            ptx::mbar_wait_inl(bar(full0, k), ((uint32_t)last_use[k] / npairs) & 1, &no_abort);
+      }
+    } else if (warp == kWarpMma || warp == kWarpPV) {
+      // ------------------------------------------------------------------ MMA issuers
+      // One thread issues the S^T MMAs (warp 9), another the P.V MMAs (warp 11): each walks the
+      // tiles in order and waits (bounded) on its own barriers, and the two overlap the per-issue
+      // work that surrounds the MMAs.  They touch disjoint tensor memory (S^T buffers, O^T) and
+      // shared memory (K ring and query rows, V ring and P^T); P.V(j) needs P^T(j), which the
+      // softmax warps publish only after loading S^T(j).  S^T(j) overwrites the buffer of
+      // S^T(j - 2), which the softmax warps release as soon as they have loaded it, so S^T(j + 2)
+      // can go out while the softmax of tile j runs.
+      if (lane == 0) {
+        const bool is_s = (warp == kWarpMma);
+        TileCursor c;
+        c.init(a);
+        // P^T as B: MN-major with 64-byte swizzle, 8 keys per 512-byte atom
+        const uint64_t bd_p = ptx::smem_desc_sw64(pbase, 16, 512);
+        uint32_t issued = 0;
+        for (; c.ok; c.advance(a)) {
+          if (is_s) {
+            const uint32_t pair = c.gt % kPairsK, ph = (c.gt / kPairsK) & 1;
+            const int qb = c.pq & 1;
+            if (c.gt >= 2) ptx::mbar_wait(bar(kBarSFree, c.gt & 1), ((c.gt - 2) >> 1) & 1, abort_flag);
+            if (c.j == 0) ptx::mbar_wait(bar(kBarQFull, qb), (c.pq >> 1) & 1, abort_flag);
+            ptx::mbar_wait(bar(kBarKFull, pair), ph, abort_flag);
+            if (*abort_flag) break;
+            ptx::tc_fence_after();
+            const uint32_t d_tmem = tmem + kColS + (c.gt & 1) * kN;
+            // K tile as A (K-major: the keys on the lanes, groups of 8 keys 2048 bytes apart),
+            // the rows as B (K-major); 16 d per k-step: 32 bytes within the 128-byte atom rows,
+            // the d-halves 1024 bytes apart
+            const uint64_t a0 = ptx::smem_desc_sw128(ring(0, pair), 16, kGroupBytes);
+            const uint64_t a1 = ptx::smem_desc_sw128(ring(0, pair) + 1024, 16, kGroupBytes);
+            const uint64_t b0 = ptx::smem_desc_sw128(qbuf(qb, 0), 16, 1024);
+            const uint64_t b1 = ptx::smem_desc_sw128(qbuf(qb, 1), 16, 1024);
+#pragma unroll
+            for (int k = 0; k < kD / 16; ++k) {
+              const uint64_t off = (uint64_t)((k & 3) * 2);
+              ptx::mma_bf16_ss(d_tmem, (k < 4 ? a0 : a1) + off, (k < 4 ? b0 : b1) + off, kIdescS,
+                               k > 0 ? 1u : 0u);
+            }
+            ptx::mma_commit(bar(kBarSFull, c.gt & 1));
+            ptx::mma_commit(bar(kBarKEmpty, pair));
+            // the pass's last S^T read of its rows: the buffer may be refilled
+            if (c.j == c.p.m.ntiles - 1) ptx::mma_commit(bar(kBarQEmpty, qb));
+          } else {
+            const uint32_t pair = c.gt % kPairsV, ph = (c.gt / kPairsV) & 1;
+            if (c.j == 0) ptx::mbar_wait(bar(kBarOFree, 0), (c.pq & 1) ^ 1, abort_flag);
+            ptx::mbar_wait(bar(kBarPFull, 0), c.gt & 1, abort_flag);
+            ptx::mbar_wait(bar(kBarVFull, pair), ph, abort_flag);
+            if (*abort_flag) break;
+            ptx::tc_fence_after();
+            const Meta &m = c.p.m;
+            const int jj = c.j;
+            const int ksteps = (jj < m.ncache) ? (min(kTK, m.npages * kPage - jj * kTK) / 16)
+                                               : kNewRows / 16;
+            // V^T as A: MN-major (D on the lanes, d-halves 1024 bytes apart, groups of 8 keys
+            // 2048 apart); fully unrolled k-steps with compile-time descriptor offsets (16 keys:
+            // 4096 bytes of V, 1024 of P^T)
+            const uint64_t ad0 = ptx::smem_desc_sw128(ring(1, pair), 1024, kGroupBytes);
+            const uint32_t acc0 = jj > 0 ? 1u : 0u;
+            if (ksteps == kTK / 16) {
+#pragma unroll
+              for (int k = 0; k < kTK / 16; ++k)
+                ptx::mma_bf16_ss(tmem + kColO, ad0 + (uint64_t)(k * 256), bd_p + (uint64_t)(k * 64),
+                                 kIdescPV, k > 0 ? 1u : acc0);
+            } else if (ksteps == kPage / 16) {
+#pragma unroll
+              for (int k = 0; k < kPage / 16; ++k)
+                ptx::mma_bf16_ss(tmem + kColO, ad0 + (uint64_t)(k * 256), bd_p + (uint64_t)(k * 64),
+                                 kIdescPV, k > 0 ? 1u : acc0);
+            } else {
+              ptx::mma_bf16_ss(tmem + kColO, ad0, bd_p, kIdescPV, acc0);
+            }
+            ptx::mma_commit(bar(kBarODone, 0));
+            ptx::mma_commit(bar(kBarVEmpty, pair));
+          }
+          ++issued;
+        }
+        // every MMA this thread issued has completed before the CTA releases shared memory and
+        // TMEM, also after an abort (each issuer drains through its own barrier)
+        if (issued > 0) {
+          const uint32_t drain = bar(kBarDrain, is_s ? 0 : 1);
+          ptx::mma_commit(drain);
+          volatile int no_abort = 0;
+          ptx::mbar_wait(drain, 0, &no_abort);
+        }
       }
     }
   } else {
+    ptx::setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax + epilogue
     const int q = warp & 3, hf = warp >> 2;
     const int kk = q * 32 + lane;  // key of the tile on this thread's TMEM lane (and d of O^T)
@@ -654,7 +665,7 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
     // before refilling the buffer of the pass with index p: the S^T MMAs of pass p - 2, its
     // previous user, are done
     auto q_wait_empty = [&](int p) {
-      if (p >= 2) ptx::mbar_wait(bar(kBarQEmpty, p & 1), ((p >> 1) - 1) & 1, abort_flag);
+      if (p >= 2) ptx::mbar_wait_inl(bar(kBarQEmpty, p & 1), ((p >> 1) - 1) & 1, abort_flag);
     };
 
     PassIter pit;
@@ -704,7 +715,7 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
         // valid keys: the tile's pages that belong to this piece, cut at the cache length
         const int vk = cache_tile ? min(min(2, m.npages - 2 * j) * kPage, m.n - (ta + 2 * j) * kPage)
                                   : m.Q;
-        ptx::mbar_wait(bar(kBarSFull, gt_ & 1), (gt_ >> 1) & 1, abort_flag);
+        ptx::mbar_wait_inl(bar(kBarSFull, gt_ & 1), (gt_ >> 1) & 1, abort_flag);
         ptx::tc_fence_after();
         softmax_tile(a, mref, lpart, tmem, lane_base, gaux, aux, abort_flag, gt_, vk, cache_tile,
                      kk, q, hf, lane, nr, kk * G - r0, pbase, j == 0);
@@ -713,7 +724,7 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
         const int vrows = cache_tile ? min(kTK, (vk + kPage - 1) / kPage * kPage) : kNewRows;
         if (vk < vrows) {
           const uint32_t pair = gt_ % kPairsV;
-          ptx::mbar_wait(bar(kBarVFull, pair), (gt_ / kPairsV) & 1, abort_flag);
+          ptx::mbar_wait_inl(bar(kBarVFull, pair), (gt_ / kPairsV) & 1, abort_flag);
           for (int idx = tid; idx < (vrows - vk) * 16; idx += kSoftmaxThreads) {
             const uint32_t row = vk + idx / 16, half = (idx % 16) / 8, c = idx % 8;
             st_shared_v4(ring(1, pair) + (row >> 3) * kGroupBytes + half * 1024 + (row & 7) * 128 +
@@ -750,7 +761,7 @@ attn_tk_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constan
         }
         lpart[0] += __shfl_xor_sync(0xffffffffu, lpart[0], 1);
         if ((lane & 1) == 0) ls[q * kRH + (lane >> 1)] = lpart[0];
-        ptx::mbar_wait(bar(kBarODone, 0), (gt + m.ntiles - 1) & 1, abort_flag);
+        ptx::mbar_wait_inl(bar(kBarODone, 0), (gt + m.ntiles - 1) & 1, abort_flag);
         ptx::tc_fence_after();
       }
       if (tid == 0 && !whole && last_pass) {  // 2: merge at once (read after the next barrier)

@@ -230,6 +230,15 @@ int dspark_verify_attn(const void *q, const void *k_new, const void *v_new, cons
     if (cudaFuncSetAttribute(tk::attn_tk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)tk::kSmemBytes) != cudaSuccess)
       return DSPARK_ECUDA;
+    // the kernel splits its register pool across warpgroups (setmaxnreg): the pool it is launched
+    // with, the compiled registers per thread x threads, must hold the split, or the increase
+    // would wait for registers that never come free
+    {
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, tk::attn_tk_kernel) != cudaSuccess) return DSPARK_ECUDA;
+      if (fa.numRegs < tk::kRegsLaunch || fa.maxThreadsPerBlock < tk::kThreads)
+        return DSPARK_EUNSUPPORTED;
+    }
     // programmatic stream serialisation: the kernel's prologue may overlap the previous kernel
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(sms);

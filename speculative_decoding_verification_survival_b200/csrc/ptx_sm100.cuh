@@ -55,11 +55,10 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// The polling loop of mbar_wait, out of line: a wait whose phase has already completed then
-// costs one try_wait and a branch (inlined, the loop's control flow costs every call about
-// ten times that).
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
-                                            volatile int *abort_flag, long long limit_cycles) {
+// The polling loop of a bounded wait, behind its first try_wait: give up once the CTA's abort
+// word is set or after limit_cycles, setting the word and recording DSPARK_DERR_TIMEOUT.
+__device__ __forceinline__ bool mbar_poll(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          long long limit_cycles) {
   if (*abort_flag) return false;
   const long long t0 = clock64();
   while (true) {
@@ -72,12 +71,28 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
     }
   }
 }
+// The same loop out of line: a wait whose phase has already completed then costs one try_wait
+// and a branch.  Inlined into a tight issue loop (a thread issuing MMAs between waits) the
+// loop's code slows every pass of it several-fold.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
+                                            volatile int *abort_flag, long long limit_cycles) {
+  return mbar_poll(bar, parity, abort_flag, limit_cycles);
+}
 // Wait for the phase with the given parity to complete; bounded.  `abort_flag` is the CTA's
 // shared abort word: once it is set, a wait whose phase has not completed returns false at once.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                           long long limit_cycles = kWaitLimitCycles) {
   if (__builtin_expect(mbar_try_wait(bar, parity), 1)) return true;
   return mbar_wait_slow(bar, parity, abort_flag, limit_cycles);
+}
+// mbar_wait with the loop inlined.  Code that runs with more registers than the kernel was
+// launched with (after setmaxnreg.inc) cannot call the out-of-line loop, and a producer that
+// waits for a free slot reacts sooner to it inlined.
+__device__ __forceinline__ bool mbar_wait_inl(uint32_t bar, uint32_t parity,
+                                              volatile int *abort_flag,
+                                              long long limit_cycles = kWaitLimitCycles) {
+  if (__builtin_expect(mbar_try_wait(bar, parity), 1)) return true;
+  return mbar_poll(bar, parity, abort_flag, limit_cycles);
 }
 
 // ---- fences / named barriers ----------------------------------------------------------------
@@ -201,6 +216,21 @@ __device__ __forceinline__ void grid_dependency_wait() {
 // Allow the next programmatically dependent launch in the stream to be scheduled.
 __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---- per-warpgroup register reallocation ------------------------------------------------------
+// Every warp of a warpgroup executes the same one.  An increase waits until the registers are
+// free in the CTA's pool (the launch's registers per thread x threads), so the split of that pool
+// across warpgroups must add up to no more than it.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "register count");
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "register count");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ---- Ampere-style asynchronous global -> shared copies (16 B, L2 only) --------------------

@@ -26,8 +26,8 @@ def test_summary_parses_nvidia_smi_lines():
              "1770, 1965, 985.50, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
              "garbage line", ""]
     s = _sampler(lines)
-    assert s == {"sm_mhz": 1785.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
-                 "samples": 3, "sufficient": False}
+    assert s == {"sm_mhz": 1785.0, "sm_max_mhz": 1965.0, "power_w": 985.5,
+                 "reasons": ["sw_power_cap"], "samples": 3, "sufficient": False}
     assert _sampler([]) is None
     s = _sampler(["1500, 1965, 700, 0x8, Not Active, Active, Not Active, Not Active"])
     assert s["reasons"] == ["hw_thermal_slowdown"]
