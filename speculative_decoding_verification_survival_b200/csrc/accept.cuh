@@ -22,6 +22,9 @@
 //                          cluster over its own run of chunks; the chunk sums are gathered
 //                          through distributed shared memory and the threshold u * Z picks the
 //                          chunk; pass 2 re-reads that chunk and scans it, in the CTA owning it.
+//                          For bf16 rows pass 1 forms the exponent arguments two at a time in
+//                          packed floats straight from the raw 16-byte groups (the same bits as
+//                          the scalar weights), in few enough registers for four CTAs per SM.
 #pragma once
 
 #include "common.cuh"
@@ -32,6 +35,9 @@ namespace dspark {
 constexpr int kAccThreads = 256;
 constexpr int kAccWarps = kAccThreads / 32;
 constexpr int kAccChunk = kAccThreads * 8;  // elements per chunk of the inverse-CDF scan
+// CTAs of the bf16 sampled draw resident per SM (its registers are bounded for that): the host
+// sizes the draw's clusters so that the whole grid fits at once where it can
+constexpr int kAccFinBlocks = 4;
 
 struct RowStats {
   float m;      // row maximum
@@ -388,6 +394,53 @@ __device__ __forceinline__ double weights8(const RowPair<T> &rp, int base, int V
   return (double)s;
 }
 
+// The same sum for eight bf16 logits of a row pair taken straight from their raw 16-byte groups,
+// the exponent arguments two elements per packed-float operation.  Bit for bit what weights8
+// gives: the packed add, multiply and fused multiply-add round each lane as the scalar
+// operations do, x - y is x + (-y), and a -inf logit gives weight 0 without the clamp of
+// ExpScale::mul (c's low part is > 0 for sampled rows).  The products by 1/Z and the difference
+// p - q stay scalar with explicit rounding, so that nothing fuses them into one rounding (an
+// empty residual must stay exactly empty); the eight weights are added in index order.
+struct PackedPairConsts {
+  uint64_t hi2, lo2, nmt2, nmd2;
+};
+template <typename T>
+__device__ __forceinline__ PackedPairConsts packed_consts(const RowPair<T> &rp) {
+  PackedPairConsts k;
+  k.hi2 = ptx::f2_pack(rp.c.hi, rp.c.hi);
+  k.lo2 = ptx::f2_pack(rp.c.lo, rp.c.lo);
+  k.nmt2 = ptx::f2_pack(-rp.mt, -rp.mt);
+  k.nmd2 = ptx::f2_pack(-rp.md, -rp.md);
+  return k;
+}
+template <typename T>
+__device__ __forceinline__ float weights8_bf16_packed(const RowPair<T> &rp,
+                                                      const PackedPairConsts &k,
+                                                      const uint4 &rt, const uint4 &rd) {
+  const uint32_t wt[4] = {rt.x, rt.y, rt.z, rt.w};
+  const uint32_t wd[4] = {rd.x, rd.y, rd.z, rd.w};
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint64_t dt = ptx::f2_add(ptx::f2_pack(__uint_as_float(wt[i] << 16),
+                                                 __uint_as_float(wt[i] & 0xffff0000u)), k.nmt2);
+    float e0, e1;
+    ptx::f2_unpack(ptx::f2_fma(dt, k.lo2, ptx::f2_mul(dt, k.hi2)), e0, e1);
+    float w0 = __fmul_rn(exp2_sfu(e0), rp.invZt), w1 = __fmul_rn(exp2_sfu(e1), rp.invZt);
+    if (rp.residual) {
+      const uint64_t dd = ptx::f2_add(ptx::f2_pack(__uint_as_float(wd[i] << 16),
+                                                   __uint_as_float(wd[i] & 0xffff0000u)), k.nmd2);
+      float g0, g1;
+      ptx::f2_unpack(ptx::f2_fma(dd, k.lo2, ptx::f2_mul(dd, k.hi2)), g0, g1);
+      w0 = fmaxf(0.f, __fsub_rn(w0, __fmul_rn(exp2_sfu(g0), rp.invZd)));
+      w1 = fmaxf(0.f, __fsub_rn(w1, __fmul_rn(exp2_sfu(g1), rp.invZd)));
+    }
+    s += w0;
+    s += w1;
+  }
+  return s;
+}
+
 __device__ __forceinline__ double block_excl_scan_f64_acc(double x, double *sm) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   double incl = x;
@@ -422,7 +475,31 @@ __device__ int draw_inverse_cdf(const RowPair<T> &rp, int V, float u, double *fs
   double *all_sum = chunk_sum + nch;          // [nch + 2], every chunk, then thr and base
   const int lo = chunk_lo(nch, rank, ncl), hi = chunk_lo(nch, rank + 1, ncl);
   constexpr int kU = 4;
-  for (int ch0 = lo; ch0 < hi; ch0 += kU) {
+  if constexpr (sizeof(T) == 2) {
+    if (rp.vec) {  // bf16, V % 8 == 0, rows aligned: packed weights from the raw groups
+      const PackedPairConsts kc = packed_consts(rp);
+      for (int ch0 = lo; ch0 < hi; ch0 += kU) {
+        uint4 rt[kU], rd[kU];
+#pragma unroll
+        for (int k = 0; k < kU; ++k) {
+          const int base = (ch0 + k) * kAccChunk + tid * 8;
+          const int b = base < V ? base : 0;  // in-bounds address; a group past V weighs 0
+          rt[k] = __ldg(reinterpret_cast<const uint4 *>(rp.t + b));
+          rd[k] = rp.residual ? __ldg(reinterpret_cast<const uint4 *>(rp.d + b)) : rt[k];
+        }
+#pragma unroll
+        for (int k = 0; k < kU; ++k) {
+          if (ch0 + k < hi) {
+            const int base = (ch0 + k) * kAccChunk + tid * 8;
+            const float sf = base < V ? weights8_bf16_packed(rp, kc, rt[k], rd[k]) : 0.f;
+            const double sd = warp_sum((double)sf);
+            if (lane == 0) part[warp * nch + ch0 + k] = sd;
+          }
+        }
+      }
+    }
+  }
+  for (int ch0 = lo; ch0 < hi && !(sizeof(T) == 2 && rp.vec); ch0 += kU) {
     float xt[kU][8], xd[kU][8];
     if (rp.vec) {  // V % 8 == 0, rows aligned: a group is either wholly inside or past the end
       Raw8<T> rt[kU], rd[kU];
@@ -531,7 +608,7 @@ __device__ int draw_inverse_cdf(const RowPair<T> &rp, int V, float u, double *fs
 // the correction / bonus draw.  CTA 0 writes the outputs except a drawn token, which the CTA
 // owning its chunk writes.
 template <typename T, bool GREEDY>
-__global__ void __launch_bounds__(kAccThreads)
+__global__ void __launch_bounds__(kAccThreads, (sizeof(T) == 2 && !GREEDY) ? kAccFinBlocks : 2)
 accept_finalize_kernel(const T *__restrict__ target, const T *__restrict__ draft, int V, int R,
                        int K, int T_cap, const int32_t *__restrict__ draft_tokens,
                        const int32_t *__restrict__ verify_len,

@@ -305,15 +305,16 @@ int dspark_accept(const void *target_logits, const void *draft_logits, int dtype
   const int nrows = T_cap + R * K;
   const size_t fin_smem = accept_finalize_smem(V);
   if (fin_smem > 227 * 1024) return DSPARK_EUNSUPPORTED;
-  // CTAs per request for the draw: as many as keep the whole grid resident at two CTAs per SM
-  // (the sampled kernel's registers allow two), at most 8 (the portable cluster size), never
-  // more than the row has chunks
+  // CTAs per request for the draw: as many as keep the whole grid resident (kAccFinBlocks CTAs
+  // per SM for bf16 rows, two for f32), at most 8 (the portable cluster size), never more than
+  // the row has chunks
   int ncl = 1;
   if (!greedy) {
     const int sms = sm_count();
     if (sms <= 0) return DSPARK_ECUDA;
     const int nch = (V + kAccChunk - 1) / kAccChunk;
-    ncl = std::max(1, std::min({8, nch, 2 * sms / R}));
+    const int per_sm = dtype == DSPARK_BF16 ? kAccFinBlocks : 2;
+    ncl = std::max(1, std::min({8, nch, per_sm * sms / R}));
   }
   auto run = [&](auto tag) -> int {
     using T = decltype(tag);
