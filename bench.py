@@ -134,13 +134,13 @@ class ClockSampler:
 # any change to those voids the figure.  Entries: (sha, bytes, algorithmic bytes of the capture);
 # a capture of another size of the same workload is scaled by algorithmic bytes.
 NCU_TRAFFIC = {
-    # one launch of the full workload (a 1-pass capture): 22 411 018 496 B read + 37 052 416 B
+    # one launch of the full workload (a 1-pass capture): 22 410 693 632 B read + 37 202 176 B
     # written, 22 324 592 640 algorithmic bytes
-    "lognormal-1024req": ("6c751188c09a7f55360fe03ab670a01ae474a9aa", 22448070912, 22324592640),
-    "lognormal-1024req-greedy": ("6c751188c09a7f55360fe03ab670a01ae474a9aa", 22448070912,
+    "lognormal-1024req": ("e840b321bde13108a61c6304d457b563a463b647", 22447895808, 22324592640),
+    "lognormal-1024req-greedy": ("e840b321bde13108a61c6304d457b563a463b647", 22447895808,
                                  22324592640),
-    # 626 557 696 B read + 4 208 128 B written, 621 088 768 algorithmic bytes
-    "qwen3-4b-64req": ("6c751188c09a7f55360fe03ab670a01ae474a9aa", 630765824, 621088768),
+    # 626 555 904 B read + 4 280 064 B written, 621 088 768 algorithmic bytes
+    "qwen3-4b-64req": ("e840b321bde13108a61c6304d457b563a463b647", 630835968, 621088768),
 }
 
 ATTN_SOURCES = ("attn_tk.cuh", "attn_common.cuh", "ptx_sm100.cuh", "common.cuh", "dspark.cu")
