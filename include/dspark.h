@@ -204,9 +204,11 @@ int dspark_verify_attn_plan(const int32_t *kv_len, const int32_t *q_offsets,
  *            rows of D elements runs on the tensor cores (tcgen05 + TMA); every other shape
  *            runs on CUDA cores.  The tensor-core path takes each request's offset, token count
  *            and validity from the records of the last dspark_verify_attn_plan (which checked
- *            the markers); the CUDA-core path checks the markers itself.  A bounded in-kernel
- *            wait that expires (a stalled copy or tensor-core pipe, after about 2 s) sets
- *            DSPARK_DERR_TIMEOUT and leaves the output undefined.
+ *            the markers); the CUDA-core path checks the markers itself.  The tensor-core kernel
+ *            splits its register pool across warp roles; a build whose compiled register count
+ *            cannot hold that split is refused with DSPARK_EUNSUPPORTED before any launch.
+ *            A bounded in-kernel wait that expires (a stalled copy or tensor-core pipe, after
+ *            about 2 s) sets DSPARK_DERR_TIMEOUT and leaves the output undefined.
  * Limits: 1 <= D <= 256 with D % 8 == 0, Hq % Hkv == 0, (Hq/Hkv)*(K+1) <= 128.
  */
 int dspark_verify_attn(const void *q, const void *k_new, const void *v_new,
