@@ -33,14 +33,22 @@ STREAM_DRAFT_VOCAB = 3
 
 
 def bf16_round(x: np.ndarray) -> np.ndarray:
-    """Round float64 values to the nearest bfloat16 (ties to even), returned as float64."""
-    f = np.asarray(x, dtype=np.float64).astype(np.float32)
-    # the float32 rounding first is exact for values whose float64 -> bf16 rounding is decided
-    # by more than float32 precision; values within float32 rounding of a bf16 tie are rare
-    b = f.view(np.uint32).astype(np.uint64)
-    lsb = (b >> np.uint64(16)) & np.uint64(1)
-    r = (b + np.uint64(0x7FFF) + lsb) & np.uint64(0xFFFF0000)
-    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+    """Round float64 values to the nearest bfloat16 (ties to even), returned as float64.
+
+    One rounding of the float64 value: bfloat16 keeps 8 significant bits down to 2^-126 and a
+    fixed quantum of 2^-133 below it (subnormals); a value at or past the midpoint between the
+    largest finite bfloat16, (2 - 2^-7) * 2^127, and 2^128 becomes infinite.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = x.copy()
+    fin = np.isfinite(x)
+    xf = x[fin]
+    _, e = np.frexp(xf)                        # xf = m * 2^e, 1/2 <= |m| < 1
+    q = np.ldexp(1.0, np.maximum(e, -125) - 8)  # the bfloat16 quantum at xf's binade
+    r = np.round(xf / q) * q                   # exact scaling, round half to even
+    r[np.abs(r) >= 2.0 ** 128] = np.inf * np.sign(r[np.abs(r) >= 2.0 ** 128])
+    out[fin] = r
+    return out
 
 
 def gumbel_uniforms(round_idx: int, r: int, k: int, V: int, seed: int = 0) -> np.ndarray:

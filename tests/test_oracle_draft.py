@@ -7,10 +7,33 @@ from oracle.draft import bf16_round, gumbel_uniforms, markov_draft_ref
 
 
 def test_bf16_rounding_matches_the_library_cast():
+    # float32 inputs: the library's float32 -> bfloat16 cast is then a single rounding too
     rng = np.random.default_rng(0)
-    x = rng.normal(0, 10, size=10000)
-    want = torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).double().numpy()
-    np.testing.assert_array_equal(bf16_round(x), want)
+    x32 = np.concatenate([rng.normal(0, 10, size=10000), rng.normal(0, 1e-38, size=1000),
+                          [0.0, -0.0, 3.38e38, -3.39e38, 1e-45]]).astype(np.float32)
+    want = torch.from_numpy(x32).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(bf16_round(x32.astype(np.float64)), want)
+
+
+def test_bf16_rounding_is_one_rounding_of_the_float64_value():
+    e = 2.0 ** -8                                   # half a bfloat16 ulp at 1
+    # just above the tie by less than a float32 ulp: a rounding through float32 would land on
+    # the tie and go to the even neighbour 1; the float64 value rounds up
+    assert bf16_round(np.array([1 + e + 2.0 ** -30]))[0] == 1 + 2 * e
+    assert bf16_round(np.array([-(1 + e + 2.0 ** -30)]))[0] == -(1 + 2 * e)
+    # exact ties go to the even neighbour
+    assert bf16_round(np.array([1 + e]))[0] == 1.0
+    assert bf16_round(np.array([1 + 3 * e]))[0] == 1 + 4 * e
+    # subnormal quantum 2^-133: ties to even there too
+    assert bf16_round(np.array([2.0 ** -134]))[0] == 0.0
+    assert bf16_round(np.array([3 * 2.0 ** -134]))[0] == 2.0 ** -132
+    # the largest finite value and overflow at the midpoint past it
+    big = (2 - 2.0 ** -7) * 2.0 ** 127
+    assert bf16_round(np.array([big]))[0] == big
+    assert bf16_round(np.array([(2 - 2.0 ** -8) * 2.0 ** 127 - 2.0 ** 100]))[0] == big
+    assert bf16_round(np.array([(2 - 2.0 ** -8) * 2.0 ** 127]))[0] == np.inf
+    assert np.isnan(bf16_round(np.array([np.nan]))[0])
+    assert bf16_round(np.array([-np.inf]))[0] == -np.inf
 
 
 def test_forced_transition_walks_the_vocabulary():
