@@ -68,6 +68,27 @@ def test_first_token_follows_target(name):
     _chi2_ok(counts, target_probs(zt[0]))
 
 
+def test_first_token_follows_the_tempered_target():
+    """At temperature tau the verifier's distribution is p = softmax(z_target / tau) and the
+    drafts come from q = softmax(z_draft / tau): the first emitted token must follow p, not
+    softmax(z_target) (the lognormal workloads sample at tau = 0.7)."""
+    tau, V = 0.7, 8
+    g = np.random.default_rng(21)
+    zt = np.tile(g.normal(0, 1.0, V).astype(np.float32), (K + 1, 1))
+    zd = np.tile(g.normal(0, 1.0, V).astype(np.float32), (K, 1))
+    rng = np.random.default_rng(5)
+    counts = np.zeros(V, dtype=np.int64)
+    n, chunk = 300_000, 100_000
+    for c0 in range(0, n, chunk):
+        tr = build_trials(zt, zd / tau, 5, chunk, rng, round_idx=11, r_base=c0)
+        tr["draft_logits"] = np.broadcast_to(zd, tr["draft_logits"].shape)
+        counts += np.bincount(_run(tr, tau)["out_tokens"][:, 0], minlength=V)
+    _chi2_ok(counts, target_probs(zt[0] / tau))
+    # the untempered distribution is far from what was drawn
+    exp1 = target_probs(zt[0]) * counts.sum()
+    assert chisquare(counts, exp1).pvalue < 1e-6
+
+
 def test_first_token_v32_position_dependent():
     rng = np.random.default_rng(42)
     V = 32
