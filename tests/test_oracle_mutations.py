@@ -84,6 +84,14 @@ def _flatten_late(verify_len, kv_len):
     return q_offsets, markers
 
 
+_schedule = O_sched.schedule_ref
+
+
+def _objective_one_late(conf, kv_len, t_ms, T_cap):   # f(n) over the time of n + 1 tokens
+    t = np.asarray(t_ms, dtype=np.float64)
+    return _schedule(conf, kv_len, np.concatenate([t[1:], t[-1:]]), T_cap)
+
+
 SCHEDULE_MUTANTS = {
     "survival without its first factor": ("survival_ref", _survival_exclusive),
     "survival without the product": ("survival_ref", _survival_no_product),
@@ -91,6 +99,7 @@ SCHEDULE_MUTANTS = {
     "ties broken by request before position": ("candidate_order", _order_r_before_k),
     "confidences one round old": ("lagged_round", lambda i: max(i - 1, 0)),
     "markers one position late": ("flatten_ref", _flatten_late),
+    "objective over the next batch size's time": ("schedule_ref", _objective_one_late),
 }
 
 
@@ -142,8 +151,13 @@ def _transposed_q(a):                 # query heads of a group read in reverse o
     return dict(a, q=q[:, ::-1, :].copy())
 
 
+def _one_key_short(a):
+    return dict(a, kv_len=np.maximum(np.asarray(a["kv_len"]) - 1, 0))
+
+
 ATTENTION_MUTANTS = {
     "scale dropped": _no_scale,
+    "one cached key too few": _one_key_short,
     "keys and values swapped": _swap_kv,
     "block table ignored": _logical_pages,
     "query heads reversed": _transposed_q,
@@ -231,12 +245,13 @@ def test_accept_pins_catch(monkeypatch, mutant):
 _commit = O_kv.kv_commit_ref
 
 
-def _commit_with(da=0, swap=False):
+def _commit_with(da=0, swap=False, late=0):
     def fn(k_new, v_new, caches, block_table, kv_len, q_offsets, accepted_len, K, T_cap):
         a = np.asarray(accepted_len) + da
         if swap:
             k_new, v_new = v_new, k_new
-        return _commit(k_new, v_new, caches, block_table, kv_len, q_offsets, a, K, T_cap)
+        return _commit(k_new, v_new, caches, block_table, np.asarray(kv_len) + late, q_offsets,
+                       a, K, T_cap)
     return fn
 
 
@@ -244,6 +259,7 @@ COMMIT_MUTANTS = {
     "one token too few": _commit_with(da=-1),
     "one token too many": _commit_with(da=+1),
     "keys and values swapped": _commit_with(swap=True),
+    "written one position late": _commit_with(late=1),
 }
 
 COMMIT_PINS = [
@@ -267,6 +283,7 @@ CALIBRATION_MUTANTS = {
     "logit multiplied by the temperature": ("calibrate_ref", lambda l, t: _calibrate(l, 1.0 / np.asarray(t, np.float64))),
     "fit returns 1 / temperature": ("fit_temperature_ref", lambda *a: 1.0 / _fit(*a)),
     "outcomes one position late": ("outcomes_from_accept", lambda *a: np.roll(_outcomes(*a), 1, axis=1)),
+    "logit sign flipped": ("calibrate_ref", lambda l, t: _calibrate(-np.asarray(l), t)),
 }
 
 CALIBRATION_PINS = [
@@ -293,6 +310,8 @@ DRAFT_MUTANTS = {
         B, E, U, np.zeros_like(np.asarray(x0)), tau, round_idx, seed),
     "transition transposed": lambda B, E, U, x0, tau, round_idx, seed=0: _draft(
         B, np.asarray(U).T, np.asarray(E).T, x0, tau, round_idx, seed),
+    "previous token off by one": lambda B, E, U, x0, tau, round_idx, seed=0: _draft(
+        B, E, U, (np.asarray(x0) + 1) % np.asarray(B).shape[-1], tau, round_idx, seed),
 }
 
 DRAFT_PINS = [
